@@ -1,0 +1,375 @@
+"""Benchmark of one absorbed-MLA decode step (one layer) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference] [--config v3]
+
+A step is the whole decode path over one batch: mla_cache_append (the batch's new tokens),
+mla_absorb_q, mla_decode (schedule + split-KV attention + log-sum-exp combine) and
+mla_out_proj.  The default workload is the DeepSeek-V3-shaped single-layer decode (n_h=128,
+d_h=128, d_c=512, d_R=64, bf16 cache, batch 16, context 4096, s_q=1, 64-token pages).
+
+Timing: CUDA events on the launching stream around each step, after W warm-up steps; the L2
+is flushed (a 512 MiB write) before every timed step, outside the events.  Under torchrun
+every rank runs its own replica (weak scaling, no collective on the data path) and the
+reported time is the max over ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (test infrastructure) on the host cores, on a
+bounded sample of the same workload, and prints the same JSON line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "absorbed-MLA decode tokens/s; latent-cache GB/s & TFLOP/s vs B200 roofline"
+WORKLOADS = {
+    "v3": "DeepSeek-V3-shaped single layer decode: n_h=128, d_h=128, d_c=512, d_R=64, bf16 latent "
+          "cache, batch 16, uniform context 4096, s_q=1, page 64",
+    "varlen": "V3 dims, batch 64, context U[1024,16384], permuted block table, bf16",
+    "long": "V3 dims, batch 4, context 131072, per-token norms LogNormal(0,0.5), bf16",
+    "mtp_fp8": "V3 dims, batch 128, context 8192, s_q=2 causal, FP8 e4m3 content + bf16 RoPE key",
+}
+FLUSH_BYTES = 512 << 20
+
+
+def make_workload(name: str):
+    from mla_latent_kv_mqa_b200 import workloads as W
+    if name == "v3":
+        return W.v3_decode()
+    if name == "varlen":
+        return W.varlen_decode()
+    if name == "long":
+        return W.long_decode()
+    if name == "mtp_fp8":
+        return W.mtp_fp8_decode()
+    raise SystemExit(f"unknown config {name}")
+
+
+def algorithmic(wl):
+    """Cache bytes and FLOPs of one mla_decode over the workload (per the method's definition:
+    each query row reads its visible cache rows once; 2*(d_c+d_R) + 2*d_c FLOPs per head and
+    visible token)."""
+    d = wl.dims
+    vis = np.array([int(L) - wl.s_q + i + 1 for L in wl.seq_lens for i in range(wl.s_q)], dtype=np.int64)
+    if wl.kv_dtype == "fp8":
+        bpt = d.d_c + 2 * d.d_r + 4
+    elif wl.kv_dtype == "f32":
+        bpt = 4 * (d.d_c + d.d_r)
+    else:
+        bpt = 2 * (d.d_c + d.d_r)
+    cache_bytes = int(wl.seq_lens.astype(np.int64).sum()) * bpt  # each cached row read once per step
+    flops = int(vis.sum()) * 2 * d.n_h * ((d.d_c + d.d_r) + d.d_c)
+    return cache_bytes, flops
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) of SM clock and throttle reasons while running, for the
+    GPU whose PCI bus id is ``bus``."""
+    Q = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, bus: int | None):
+        self.bus = bus
+        self.rows = []
+        self.error = None
+        self._p = None
+
+    def __enter__(self):
+        try:
+            self._p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                        "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except OSError as e:
+            self.error = str(e)
+            self._p = None
+        return self
+
+    def _read(self):
+        for line in self._p.stdout:
+            r = [x.strip() for x in line.split(",")]
+            if len(r) < 9:
+                continue
+            try:
+                bus = int(r[0].split(":")[1], 16)
+            except (IndexError, ValueError):
+                bus = None
+            if self.bus is None or bus == self.bus:
+                self.rows.append(r)
+
+    def __exit__(self, *a):
+        if self._p:
+            self._p.terminate()
+            try:
+                _, err = self._p.communicate(timeout=5)
+                if not self.rows and err:
+                    self.error = err.strip()[:200]
+            except subprocess.TimeoutExpired:
+                self._p.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0,
+                    "error": self.error}
+        num = lambda x: float(x) if x.replace(".", "", 1).isdigit() else None
+        sm = [v for v in (num(r[1]) for r in self.rows) if v is not None]
+        mx = [v for v in (num(r[2]) for r in self.rows) if v is not None]
+        pw = [v for v in (num(r[3]) for r in self.rows) if v is not None]
+        reasons = sorted({self.NAMES[i] for r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None, "reasons": reasons, "samples": len(self.rows)}
+
+
+def cpu_baseline(wl, budget_s: float = 12.0):
+    """The fp64 oracle (absorbed mode), as it stands, on a bounded sample of the workload:
+    whole sequences (all heads, all visible tokens) until ``budget_s`` is spent."""
+    from oracle import oracle as orc
+    from tests.harness import oracle_ref
+    orc.build()
+    t0 = time.perf_counter()
+    n_seq = 0
+    for b in range(wl.B):
+        oracle_ref(wl, orc, seqs=[b])
+        n_seq += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": n_seq * wl.s_q / dt, "unit": "tokens/s", "cores": orc.num_threads(), "kind": "oracle",
+            "sample": f"{n_seq} of {wl.B} sequences, all {wl.dims.n_h} heads, fp64 absorbed mode, {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = make_workload(args.config)
+    from oracle import oracle as orc
+    from tests.harness import oracle_ref
+    orc.build()
+    budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    times, toks = [], 0
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        n = 0
+        for b in range(wl.B):
+            oracle_ref(wl, orc, seqs=[b])
+            n += 1
+            if time.perf_counter() - t0 > budget:
+                break
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+            toks += n * wl.s_q
+    total = float(sum(times))
+    value = toks / total
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOADS[args.config], "sample": "per step: whole "
+                                            "sequences in order until the step's CPU budget is spent"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": orc.num_threads(), "kind": "oracle",
+                             "sample": f"{toks} query tokens over {len(times)} steps of up to {budget:.1f} s"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_mine(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    from mla_latent_kv_mqa_b200 import build
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    from mla_latent_kv_mqa_b200 import layer as Lyr
+    from mla_latent_kv_mqa_b200 import native as N
+    from tests.harness import GpuRun
+
+    wl = make_workload(args.config)
+    run = GpuRun(wl, dev=dev)
+    run.fill_cache()
+    L = run.layer
+    B, s_q, T = wl.B, wl.s_q, wl.T
+    # this step's new tokens: the last s_q cache rows of every sequence (rewritten every step)
+    idx = np.concatenate([np.arange(wl.ctx_off[b + 1] - s_q, wl.ctx_off[b + 1]) for b in range(B)])
+    tok_seq = run.tok_seq[torch.from_numpy(idx).to(dev)].contiguous()
+    tok_pos = run.tok_pos[torch.from_numpy(idx).to(dev)].contiguous()
+    c_new = run.c_kv[torch.from_numpy(idx).to(dev)].contiguous()
+    k_new = run.k_r[torch.from_numpy(idx).to(dev)].contiguous()
+    q_abs = torch.empty((T, wl.dims.n_h, wl.dims.row), dtype=run.q_c.dtype, device=dev)
+    o_lat = torch.empty((T, wl.dims.n_h, wl.dims.d_c), dtype=torch.float32, device=dev)
+    lse = torch.empty((T, wl.dims.n_h), dtype=torch.float32, device=dev)
+    o = torch.empty((T, wl.dims.n_h, wl.dims.d_h), dtype=torch.float32, device=dev)
+    ws = L.workspace(B, s_q, run.max_seq_len)
+    decode_launches = 3 if (wl.kv_dtype == "bf16" and wl.dims.n_h == 128) else 2
+    launches_per_step = 1 + 1 + decode_launches + 1
+
+    def step(_unused=None, tok=(tok_seq, tok_pos, c_new, k_new), qin=(run.q_c, run.q_r, run.q_pos), out=o):
+        L.append(run.cache, tok[2], tok[3], tok[0], tok[1], run.block_table)
+        L.absorb(qin[0], qin[1], qin[2], out=q_abs)
+        L.decode(run.cache, q_abs, run.block_table, run.seq_lens, s_q, run.max_seq_len, o_lat=o_lat, lse=lse)
+        L.out_proj(o_lat, "f32", out=out)
+
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    pin = lambda x: x.cpu().pin_memory()
+    h_in = [pin(x) for x in (tok_seq, tok_pos, c_new, k_new, run.q_c, run.q_r, run.q_pos)]
+    d_in = [torch.empty_like(x) for x in (tok_seq, tok_pos, c_new, k_new, run.q_c, run.q_r, run.q_pos)]
+    h_out = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in h_in)
+    d2h = h_out.numel() * h_out.element_size()
+
+    def decode_only():
+        L.decode(run.cache, q_abs, run.block_table, run.seq_lens, s_q, run.max_seq_len, o_lat=o_lat, lse=lse)
+
+    def e2e_step():
+        for h, d_ in zip(h_in, d_in):
+            d_.copy_(h, non_blocking=True)
+        step(None, tok=tuple(d_in[:4]), qin=tuple(d_in[4:]))
+        h_out.copy_(o, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):  # eager warm-up (also sets up kernel attributes)
+            flush.fill_(1)
+            step()
+            e2e_step()
+        stream.synchronize()
+        if N.mla_get_last_device_error() != 0:
+            raise SystemExit("device error during warm-up")
+        g_step, g_dec, g_e2e = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_step, stream=stream):
+            step()
+        with torch.cuda.graph(g_dec, stream=stream):
+            decode_only()
+        with torch.cuda.graph(g_e2e, stream=stream):
+            e2e_step()
+        for _ in range(max(args.warmup, 3)):  # graph warm-up
+            flush.fill_(2)
+            g_step.replay()
+            g_dec.replay()
+            g_e2e.replay()
+        stream.synchronize()
+
+        K = args.steps
+        mk = lambda: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        ev, dev_ev, e2e_ev = mk(), mk(), mk()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        bus = torch.cuda.get_device_properties(dev).pci_bus_id
+        with ClockSampler(bus) as clk:
+            for k in range(K):
+                flush.fill_(k & 0xFF)
+                ev[k][0].record(stream)
+                g_step.replay()
+                ev[k][1].record(stream)
+                flush.fill_((k + 1) & 0xFF)
+                dev_ev[k][0].record(stream)
+                g_dec.replay()
+                dev_ev[k][1].record(stream)
+            stream.synchronize()
+            if world > 1:
+                dist.barrier()
+            # end to end through the public API: pinned host inputs in, host result out
+            for k in range(K):
+                flush.fill_(k & 0xFF)
+                e2e_ev[k][0].record(stream)
+                g_e2e.replay()
+                e2e_ev[k][1].record(stream)
+                stream.synchronize()
+                _ = float(h_out[0, 0, 0])  # the host reads the step's result
+    step_ms = sum(a.elapsed_time(b) for a, b in ev) / K
+    dec_ms = sum(a.elapsed_time(b) for a, b in dev_ev) / K
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / K
+    t = torch.tensor([step_ms, dec_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    step_ms, dec_ms, e2e_ms = float(t[0]), float(t[1]), float(t[2])
+    if N.mla_get_last_device_error() != 0:
+        raise SystemExit("device error during the timed region")
+    del g_step, g_dec, g_e2e
+
+    cache_bytes, flops = algorithmic(wl)
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        hbm_peak, tc_peak, src = peaks["hbm_gbs"], peaks["bf16_tflops"], "measured"
+    except (OSError, KeyError, ValueError):
+        hbm_peak, tc_peak, src = 6650.0, 1590.0, "fallback"
+    dec_s = dec_ms * 1e-3
+    gbs = cache_bytes / dec_s / 1e9
+    tfl = flops / dec_s / 1e12
+    bound = "hbm" if cache_bytes / (hbm_peak * 1e9) >= flops / (tc_peak * 1e12) else "tensor"
+    achieved, peak, unit = (gbs, hbm_peak, "GB/s") if bound == "hbm" else (tfl, tc_peak, "TFLOP/s")
+    tokens = T * world
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": tokens / (step_ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.kv_dtype == "bf16" else wl.kv_dtype,
+        "data": "synthetic",
+        "config": {"workload": WORKLOADS[args.config], "batch_per_gpu": B, "s_q": s_q,
+                   "context": int(wl.seq_lens.max()), "parallelism": f"replicas x{world}",
+                   "l2": "flushed before every timed step (512 MiB write outside the events)",
+                   "launch": "each step is one CUDA-graph replay of the four calls"},
+        "decode": {"kernel": "mla_decode (schedule + tcgen05 split-KV main + LSE combine)",
+                   "ms": dec_ms, "tokens_per_s": tokens / dec_s, "cache_gbs": gbs, "tflops": tfl,
+                   "frac_hbm": gbs / hbm_peak, "frac_bf16": tfl / tc_peak,
+                   "cache_bytes": cache_bytes, "flops": flops},
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "traffic": None, "peak_source": src,
+                     "kernel": "mla_decode", "algorithmic_per_launch": cache_bytes if bound == "hbm" else flops},
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "how": "CUDA graph of pinned H2D copies + the four calls + D2H of o; host reads o each step"},
+        "gpu_launches": (launches_per_step + decode_launches) * K,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
+    ap.add_argument("--config", default="v3", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_mine(args)
+
+
+if __name__ == "__main__":
+    main()

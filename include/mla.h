@@ -1,0 +1,185 @@
+/*
+ * mla.h -- C ABI of libmla: absorbed (MQA-mode) Multi-head Latent Attention decode
+ * over a paged latent KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * The method is the one of the itwiki article "멀티 헤드 잠재 어텐션"
+ * (Multi-head latent attention):
+ *   - section 구조 (structure): the cache holds the joint latent c^KV_t = W^DKV h_t
+ *     (d_c wide); keys and values are W^UK c and W^UV c with W^UK, W^UV of shape
+ *     [n_h*d_h, d_c].
+ *   - section 행렬 흡수 (matrix absorption): the score q^T W^UK c is computed as
+ *     (W^UK^T q)^T c, so each head's query is moved into the latent space and all
+ *     heads score the same cached c^KV; W^UV is applied after the weighted sum.
+ *   - section 분리 RoPE (decoupled RoPE): a per-head RoPE query q^R and one shared
+ *     RoPE key k^R_t are concatenated to the content parts; the cache stores
+ *     [c^KV_t ; k^R_t], d_c + d_R values per token; scores are divided by
+ *     sqrt(d_h + d_R) and softmaxed over the tokens j <= t.
+ *   - section 구현 (implementation): half-split RoPE, angle pos * base^(-2k/d_R).
+ * The lecture page "MHA · GQA · MQA · MLA", section "Why Projection Absorption
+ * Helps", gives the same identity q^T W_UK c_t = (W_UK^T q)^T c_t.
+ *
+ * One decode step of one layer is four calls, in this order on one stream:
+ *   mla_cache_append  -- write the new tokens' [c^KV ; RoPE(k^R)] rows into the cache
+ *   mla_absorb_q      -- q_abs = [W^UK_h^T q^C ; RoPE(q^R)]  per token and head
+ *   mla_decode        -- split-KV attention over the cache + log-sum-exp combine
+ *   mla_out_proj      -- o = W^UV_h o_lat per token and head
+ *
+ * Conventions shared by every call
+ *   Memory     The caller owns every buffer; all pointers are device pointers of one
+ *              device (the current device) unless a comment says otherwise.  The
+ *              library allocates no device memory besides one static error word per
+ *              device (see mla_get_last_device_error).
+ *   Streams    Calls only enqueue work on `stream` (NULL = the legacy default stream)
+ *              and return; results are ready in stream order.
+ *   Layouts    Row-major, contiguous, as each argument states.
+ *   Errors     Arguments are checked on the host before anything is launched; a bad
+ *              argument returns an error and launches nothing.  A launch failure
+ *              returns MLA_ERR_CUDA.  Conditions only the device can see (a block id
+ *              outside the pool, a sequence length outside its table) make the kernel
+ *              skip the offending access and set the device error word, which
+ *              mla_get_last_device_error reports.  Nothing throws across the ABI.
+ *   Softmax    The scale is 1/sqrt(d_h + d_R) (분리 RoPE section, output equation).
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so the header needs no CUDA include. */
+typedef struct CUstream_st *mla_stream_t;
+
+typedef enum {
+    MLA_OK = 0,
+    MLA_ERR_INVALID_ARG = 1,         /* null pointer, negative size, misaligned pointer */
+    MLA_ERR_UNSUPPORTED = 2,         /* dims / dtype combination not built into the library */
+    MLA_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes < mla_decode_workspace_size(...) */
+    MLA_ERR_BAD_BLOCK_TABLE = 4,     /* device saw a block id outside [0, num_blocks) */
+    MLA_ERR_BAD_SEQ_LEN = 5,         /* device saw a length < s_q or > max_blocks*page */
+    MLA_ERR_DEVICE_TIMEOUT = 6,      /* a bounded device-side wait gave up */
+    MLA_ERR_CUDA = 7                 /* a CUDA runtime call failed */
+} mla_status_t;
+
+typedef enum {
+    MLA_DTYPE_F32 = 0,
+    MLA_DTYPE_BF16 = 1,
+    MLA_DTYPE_FP8_E4M3 = 2 /* cache only: e4m3 content + per-token fp32 scale + bf16 RoPE key */
+} mla_dtype_t;
+
+/* flags */
+#define MLA_FLAG_SIMT_DECODE 1u /* run mla_decode on the CUDA-core kernel even where the
+                                   tensor-core kernel applies (cross-checks) */
+
+typedef struct {
+    int n_h;            /* heads */
+    int d_h;            /* head dim of the content query q^C and of the output o */
+    int d_c;            /* latent width of c^KV */
+    int d_r;            /* RoPE width d_R (even) */
+    int page_size;      /* tokens per cache block (64) */
+    float rope_base;    /* RoPE base (1e4) */
+    mla_dtype_t act_dtype; /* q_c, q_r, q_abs, c_kv/k_r append inputs, w_uk, w_uv: F32 or BF16 */
+    mla_dtype_t kv_dtype;  /* cache: F32, BF16 or FP8_E4M3 */
+    unsigned flags;
+} mla_dims_t;
+
+/* ----------------------------------------------------------------------------------------
+ * mla_absorb_q -- the query side of the absorbed form (행렬 흡수 section; 분리 RoPE section
+ * for q^R).  For every token t < T and head h:
+ *     q_abs[t, h, 0:d_c]         = W^UK_h^T q_c[t, h, :]      (W^UK_h = rows h*d_h .. of w_uk)
+ *     q_abs[t, h, d_c:d_c+d_r]   = RoPE(q_r[t, h, :], pos[t])
+ *   q_c   [T, n_h, d_h]   act dtype
+ *   q_r   [T, n_h, d_r]   act dtype, before rotation
+ *   pos   [T]             int32 position of each token (>= 0)
+ *   w_uk  [n_h*d_h, d_c]  act dtype (the nn.Linear(d_c, n_h*d_h) weight)
+ *   q_abs [T, n_h, d_c+d_r] act dtype, written
+ * Accumulation is fp32; the rotation angle is formed in fp64.  T == 0 is a no-op.
+ * ---------------------------------------------------------------------------------------- */
+mla_status_t mla_absorb_q(const mla_dims_t *dims, int T, const void *q_c, const void *q_r,
+                          const int32_t *pos, const void *w_uk, void *q_abs,
+                          mla_stream_t stream);
+
+/* ----------------------------------------------------------------------------------------
+ * mla_cache_append -- write new tokens into the paged latent cache (분리 RoPE section: the
+ * cache holds c^KV_t and k^R_t = RoPE(W^KR h_t), d_c + d_R values per token).
+ * Token t goes to sequence s = seq_idx[t] at position p = pos[t]:
+ *     block = block_table[s * max_blocks_per_seq + p / page_size],  slot = p % page_size.
+ *   c_kv [T, d_c] act dtype;  k_r [T, d_r] act dtype, before rotation.
+ *   BF16 / F32 cache: kv_pool [num_blocks, page_size, d_c + d_r] of that dtype, row =
+ *       [c_kv ; RoPE(k_r, p)].  kr_pool and kv_scale must be NULL.
+ *   FP8_E4M3 cache: kv_pool [num_blocks, page_size, d_c] uint8 e4m3 codes,
+ *       kr_pool [num_blocks, page_size, d_r] bf16 RoPE(k_r, p),
+ *       kv_scale [num_blocks, page_size] fp32.  Per token s = amax|c_kv|/448 computed in
+ *       fp32 (at least FLT_MIN; 1 when amax = 0); codes = e4m3(c_kv / s), nearest-even,
+ *       saturating.
+ * A token whose block id or table index is out of range is skipped and sets
+ * MLA_ERR_BAD_BLOCK_TABLE on the device.  Never reads the pool.
+ * ---------------------------------------------------------------------------------------- */
+mla_status_t mla_cache_append(const mla_dims_t *dims, int T, const void *c_kv, const void *k_r,
+                              const int32_t *seq_idx, const int32_t *pos,
+                              const int32_t *block_table, int num_seqs, int max_blocks_per_seq,
+                              int num_blocks, void *kv_pool, void *kr_pool, float *kv_scale,
+                              mla_stream_t stream);
+
+/* ----------------------------------------------------------------------------------------
+ * mla_decode_workspace_size -- bytes of device workspace mla_decode needs for B sequences of
+ * s_q queries each and sequence lengths up to max_seq_len, on the current device.  Returns 0
+ * for invalid arguments or when the current device cannot be queried.
+ * ---------------------------------------------------------------------------------------- */
+size_t mla_decode_workspace_size(const mla_dims_t *dims, int B, int s_q, int max_seq_len);
+
+/* ----------------------------------------------------------------------------------------
+ * mla_decode -- absorbed attention over the paged cache (분리 RoPE section output equation
+ * in the latent form of the 행렬 흡수 section).  Query i < s_q of sequence b (row
+ * t = b*s_q + i) sits at position P = seq_lens[b] - s_q + i and, for every head h,
+ *     s_j     = (q_abs[t,h,0:d_c] . c_j + q_abs[t,h,d_c:] . kR_j) / sqrt(d_h + d_r),  j <= P
+ *     o_lat   = sum_j softmax(s)_j c_j,       lse = ln sum_j exp(s_j)
+ * where (c_j ; kR_j) is cache row j of sequence b (FP8: c_j = e4m3(code) * scale_j).
+ * The tokens are split into segments processed in parallel; the partial results are merged
+ * exactly by a log-sum-exp combine kernel.
+ *   q_abs       [B*s_q, n_h, d_c+d_r] act dtype (from mla_absorb_q)
+ *   kv_pool, kr_pool, kv_scale: the cache, as in mla_cache_append (read only)
+ *   block_table [B, max_blocks_per_seq] int32
+ *   seq_lens    [B] int32 device array; each in [s_q, max_seq_len]
+ *   max_seq_len host-side upper bound of seq_lens (<= max_blocks_per_seq * page_size)
+ *   workspace   device scratch of workspace_bytes >= mla_decode_workspace_size(...);
+ *               its content on entry does not matter.
+ *   o_lat       [B*s_q, n_h, d_c] fp32, written
+ *   lse         [B*s_q, n_h] fp32 natural-log normaliser, written (may be NULL)
+ * Deterministic: the result depends only on the logical cache content, not on which
+ * physical blocks hold it.
+ * ---------------------------------------------------------------------------------------- */
+mla_status_t mla_decode(const mla_dims_t *dims, int B, int s_q, const void *q_abs,
+                        const void *kv_pool, const void *kr_pool, const float *kv_scale,
+                        const int32_t *block_table, int max_blocks_per_seq, int num_blocks,
+                        const int32_t *seq_lens, int max_seq_len, void *workspace,
+                        size_t workspace_bytes, float *o_lat, float *lse, mla_stream_t stream);
+
+/* ----------------------------------------------------------------------------------------
+ * mla_out_proj -- value up-projection after the aggregation (행렬 흡수 section):
+ *     o[t, h, :] = W^UV_h o_lat[t, h, :]      (d_h <- d_c; W^UV_h = rows h*d_h .. of w_uv)
+ *   o_lat [T, n_h, d_c] fp32;  w_uv [n_h*d_h, d_c] act dtype;
+ *   o     [T, n_h, d_h] of out_dtype (F32 or BF16), written.  fp32 accumulation.
+ * ---------------------------------------------------------------------------------------- */
+mla_status_t mla_out_proj(const mla_dims_t *dims, int T, const float *o_lat, const void *w_uv,
+                          void *o, mla_dtype_t out_dtype, mla_stream_t stream);
+
+/* Reads and clears the device error word of the current device.  Synchronises the device.
+ * Returns MLA_OK, MLA_ERR_BAD_BLOCK_TABLE, MLA_ERR_BAD_SEQ_LEN or MLA_ERR_DEVICE_TIMEOUT
+ * (the first condition seen since the last call), or MLA_ERR_CUDA. */
+mla_status_t mla_get_last_device_error(void);
+
+/* Static, human-readable name of a status code. */
+const char *mla_status_string(mla_status_t status);
+
+/* Library ABI version (major * 100 + minor). */
+int mla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H_ */

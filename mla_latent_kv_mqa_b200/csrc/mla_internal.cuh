@@ -1,0 +1,100 @@
+// Internal declarations of libmla (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "../../include/mla.h"
+
+namespace mla {
+
+// Device error word codes (first condition wins, see record_error).
+enum : unsigned {
+    kErrNone = 0,
+    kErrBadBlock = MLA_ERR_BAD_BLOCK_TABLE,
+    kErrBadSeqLen = MLA_ERR_BAD_SEQ_LEN,
+    kErrTimeout = MLA_ERR_DEVICE_TIMEOUT,
+};
+
+// Address of this device's error word (set up once per device by the API layer).
+unsigned *device_error_word();
+
+__device__ __forceinline__ void record_error(unsigned *err, unsigned code) {
+    if (err) atomicCAS(err, 0u, code);
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// RoPE angle tables (구현 section of the MLA article: pair k of a d_r-wide vector is rotated
+// by pos * base^(-2k/d_r)).  The angle is formed and reduced in fp64 so that positions up to
+// 2^31 keep full fp32 accuracy in cos/sin.
+__device__ __forceinline__ void rope_cos_sin(int k, int d_r, double base, int pos, float *c,
+                                             float *s) {
+    double inv_freq = pow(base, -(double)(2 * k) / (double)d_r);
+    double theta = (double)pos * inv_freq;
+    double sd, cd;
+    sincos(theta, &sd, &cd);
+    *c = (float)cd;
+    *s = (float)sd;
+}
+
+// Partial results of one split segment, shared by the decode kernels and the combine kernel.
+//   o_part [slot][n_h][d_c] fp32: sum_j exp2(s2_j - m) c_j   (not normalised)
+//   m_part [slot][n_h]      fp32: running max m in log2 units (s2 = s * log2(e)); -inf = empty
+//   l_part [slot][n_h]      fp32: sum_j exp2(s2_j - m)
+struct Partials {
+    float *o;
+    float *m;
+    float *l;
+};
+
+// ---- launchers (host) --------------------------------------------------------------------
+cudaError_t launch_append(const mla_dims_t &d, int T, const void *c_kv, const void *k_r,
+                          const int32_t *seq_idx, const int32_t *pos, const int32_t *bt,
+                          int num_seqs, int max_blocks, int num_blocks, void *kv_pool,
+                          void *kr_pool, float *kv_scale, cudaStream_t st);
+
+cudaError_t launch_absorb_q(const mla_dims_t &d, int T, const void *q_c, const void *q_r,
+                            const int32_t *pos, const void *w_uk, void *q_abs, cudaStream_t st);
+
+cudaError_t launch_out_proj(const mla_dims_t &d, int T, const float *o_lat, const void *w_uv,
+                            void *o, mla_dtype_t out_dtype, cudaStream_t st);
+
+// CUDA-core split-KV decode.  Splits every query row into n_split segments of seg_len tokens.
+struct SimtPlan {
+    int n_split;
+    int seg_len;
+};
+SimtPlan simt_plan(const mla_dims_t &d, int B, int s_q, int max_seq_len);
+size_t simt_workspace_bytes(const mla_dims_t &d, int B, int s_q, int max_seq_len);
+cudaError_t launch_decode_simt(const mla_dims_t &d, int B, int s_q, const void *q_abs,
+                               const void *kv_pool, const void *kr_pool, const float *kv_scale,
+                               const int32_t *bt, int max_blocks, int num_blocks,
+                               const int32_t *seq_lens, int max_seq_len, void *ws,
+                               float *o_lat, float *lse, cudaStream_t st);
+
+// Log-sum-exp merge of split partials.  Row r (= query row t) owns slots
+// seg_range[2r] .. seg_range[2r+1]-1 when seg_range != nullptr, else r*uniform .. r*uniform+uniform-1.
+cudaError_t launch_combine(int rows, int n_h, int d_c, Partials p, const int32_t *seg_range,
+                           int uniform, float *o_lat, float *lse, cudaStream_t st);
+
+// Tensor-core (tcgen05) decode for the DeepSeek-V3 shape.
+bool tc_supported(const mla_dims_t &d);
+size_t tc_workspace_bytes(const mla_dims_t &d, int B, int s_q, int max_seq_len);
+cudaError_t launch_decode_tc(const mla_dims_t &d, int B, int s_q, const void *q_abs,
+                             const void *kv_pool, const void *kr_pool, const float *kv_scale,
+                             const int32_t *bt, int max_blocks, int num_blocks,
+                             const int32_t *seq_lens, int max_seq_len, void *ws,
+                             size_t ws_bytes, float *o_lat, float *lse, cudaStream_t st);
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace mla

@@ -207,6 +207,18 @@ def mtp_fp8_decode(seed: int = 5, B: int = 128, L: int = 8192, s_q: int = 2) -> 
                             "bf16", rng)
 
 
+def make_decode(seed: int, seq_lens, *, s_q: int = 1, kv_dtype: str = "bf16",
+                act_dtype: str = "bf16", permute: bool = False, spare: int = 0,
+                lognormal_tokens: bool = False, dims: MLADims = V3_DIMS,
+                name: str = "custom") -> DecodeWorkload:
+    """Any decode batch with the structure of the five workloads (ragged lengths, permuted
+    tables, spare blocks, per-token norm spread)."""
+    rng = np.random.default_rng(seed)
+    ts = (lambda r, n: r.lognormal(0.0, 0.5, size=n)) if lognormal_tokens else None
+    return _decode_workload(name, dims, list(seq_lens), s_q, kv_dtype, act_dtype, rng,
+                            permute=permute, spare=spare, token_scale=ts)
+
+
 CONFIGS = {
     "toy": dict(desc="Toy MLA layer d=1024 n_h=8 d_h=64 d_c=128 d_cq=256 d_R=32, B=1, ctx 256, fp32"),
     "v3": dict(desc="DeepSeek-V3-shaped decode n_h=128 d_h=128 d_c=512 d_R=64, bf16, B=16, ctx 4096, page 64"),

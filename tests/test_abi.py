@@ -1,0 +1,79 @@
+"""The C-ABI library loads, exports every symbol include/mla.h declares, and rejects bad
+arguments on the host before touching the GPU (no compute calls here)."""
+import ctypes
+import subprocess
+
+import pytest
+
+from mla_latent_kv_mqa_b200 import build as B
+
+
+@pytest.fixture(scope="module")
+def N():
+    B.build()
+    from mla_latent_kv_mqa_b200 import native
+    return native
+
+
+def test_exports_every_declared_symbol(N):
+    names = N.declared_functions()
+    assert {"mla_absorb_q", "mla_cache_append", "mla_decode", "mla_decode_workspace_size",
+            "mla_out_proj", "mla_get_last_device_error", "mla_status_string",
+            "mla_version"} <= set(names)
+    out = subprocess.run(["nm", "-D", "--defined-only", N.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in names:
+        assert n in exported, n
+        assert hasattr(N.library(), n)
+
+
+def test_status_strings_and_version(N):
+    assert N.version() == 100
+    assert N.status_string(0) == "MLA_OK"
+    assert N.status_string(N.MLA_ERR_WORKSPACE_TOO_SMALL) == "MLA_ERR_WORKSPACE_TOO_SMALL"
+    assert N.status_string(99) == "MLA_ERR_UNKNOWN"
+
+
+def _v3(N, **kw):
+    return N.make_dims(128, 128, 512, 64, **kw)
+
+
+def test_host_argument_checks(N):
+    L = N.library()
+    d = _v3(N)
+    dp = ctypes.byref(d)
+    # null pointers with work to do
+    assert L.mla_absorb_q(dp, 4, None, None, None, None, None, None) == N.MLA_ERR_INVALID_ARG
+    # zero tokens is a no-op even with null pointers
+    assert L.mla_absorb_q(dp, 0, None, None, None, None, None, None) == N.MLA_OK
+    assert L.mla_out_proj(dp, -1, None, None, None, 0, None) == N.MLA_ERR_INVALID_ARG
+    # odd RoPE width, bad dtype
+    bad = _v3(N)
+    bad.d_r = 63
+    assert L.mla_out_proj(ctypes.byref(bad), 1, 8, 8, 8, 0, None) == N.MLA_ERR_INVALID_ARG
+    bad = _v3(N, act_dtype=N.MLA_DTYPE_FP8_E4M3)
+    assert L.mla_out_proj(ctypes.byref(bad), 1, 8, 8, 8, 0, None) == N.MLA_ERR_UNSUPPORTED
+    # fp8 cache needs the RoPE pool and the scales, and only then
+    f8 = _v3(N, kv_dtype=N.MLA_DTYPE_FP8_E4M3)
+    assert L.mla_cache_append(ctypes.byref(f8), 1, 8, 8, 8, 8, 8, 1, 1, 1, 8, None, None,
+                              None) == N.MLA_ERR_INVALID_ARG
+    assert L.mla_cache_append(dp, 1, 8, 8, 8, 8, 8, 1, 1, 1, 8, 8, None, None) == N.MLA_ERR_INVALID_ARG
+    # decode: s_q < 1, max_seq_len beyond the table, workspace too small / misaligned
+    args = [dp, 2, 0, 16, 16, None, None, 16, 4, 8, 16, 256, 256, 1 << 30, 16, 16, None]
+    assert L.mla_decode(*args) == N.MLA_ERR_INVALID_ARG
+    args = [dp, 2, 1, 16, 16, None, None, 16, 4, 8, 16, 257, 256, 1 << 30, 16, 16, None]
+    assert L.mla_decode(*args) == N.MLA_ERR_INVALID_ARG
+    simt = _v3(N, flags=N.MLA_FLAG_SIMT_DECODE)  # its size needs no device query
+    args = [ctypes.byref(simt), 2, 1, 16, 16, None, None, 16, 4, 8, 16, 256, 256, 0, 16, 16, None]
+    assert L.mla_decode(*args) == N.MLA_ERR_WORKSPACE_TOO_SMALL
+    args = [dp, 2, 1, 16, 16, None, None, 16, 4, 8, 16, 256, 8, 1 << 30, 16, 16, None]
+    assert L.mla_decode(*args) == N.MLA_ERR_INVALID_ARG
+
+
+def test_workspace_size_is_positive_and_monotone(N):
+    d = _v3(N, flags=N.MLA_FLAG_SIMT_DECODE)
+    a = N.mla_decode_workspace_size(d, 16, 1, 4096)
+    b = N.mla_decode_workspace_size(d, 64, 1, 16384)
+    assert 0 < a <= b
+    assert N.mla_decode_workspace_size(d, 4, 0, 4096) == 0
