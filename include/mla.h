@@ -73,6 +73,7 @@ typedef enum {
 /* flags */
 #define MLA_FLAG_SIMT_DECODE 1u /* run mla_decode on the CUDA-core kernel even where the
                                    tensor-core kernel applies (cross-checks) */
+#define MLA_FLAG_SIMT_PROJ 2u   /* same for mla_absorb_q and mla_out_proj */
 
 typedef struct {
     int n_h;            /* heads */

@@ -144,29 +144,74 @@ decode_simt_kernel(int s_q, int n_h, int d_c, int d_r, float scale_log2, int pag
     }
 }
 
-// Log-sum-exp merge: block per (row, head), thread per latent column.
-__global__ void combine_kernel(int n_h, int d_c, Partials p, const int32_t *__restrict__ seg_range,
-                               int uniform, float *__restrict__ o_lat, float *__restrict__ lse) {
-    const int r = blockIdx.x, h = blockIdx.y;
+// Log-sum-exp merge: block per (row, head).  The per-slot weights 2^(m_s - M) are computed once
+// into shared memory, then each thread sweeps its columns across the slots with float4 loads.
+constexpr int kCombineThreads = 128;
+constexpr int kCombineMaxSlots = 1024;
+
+__global__ void __launch_bounds__(kCombineThreads)
+combine_kernel(int n_h, int d_c, Partials p, const int32_t *__restrict__ seg_range, int uniform,
+               float *__restrict__ o_lat, float *__restrict__ lse) {
+    __shared__ float w_s[kCombineMaxSlots];
+    __shared__ float red[kCombineThreads / 32];
+    const int r = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int s0 = seg_range ? seg_range[2 * r] : r * uniform;
-    const int s1 = seg_range ? seg_range[2 * r + 1] : s0 + uniform;
-    float M = -INFINITY;
-    for (int s = s0; s < s1; ++s) M = fmaxf(M, p.m[(size_t)s * n_h + h]);
+    int s1 = seg_range ? seg_range[2 * r + 1] : s0 + uniform;
+    if (s1 - s0 > kCombineMaxSlots) s1 = s0 + kCombineMaxSlots;  // never reached: slots <= clusters + rows
+    const int S = s1 - s0;
+    float mloc = -INFINITY;
+    for (int s = tid; s < S; s += kCombineThreads) mloc = fmaxf(mloc, p.m[(size_t)(s0 + s) * n_h + h]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
+    if (lane == 0) red[wid] = mloc;
+    __syncthreads();
+    float M = red[0];
+#pragma unroll
+    for (int i = 1; i < kCombineThreads / 32; ++i) M = fmaxf(M, red[i]);
+    __syncthreads();
+    float lloc = 0.f;
+    for (int s = tid; s < S; s += kCombineThreads) {
+        const float ms = p.m[(size_t)(s0 + s) * n_h + h];
+        const float w = ms == -INFINITY ? 0.f : exp2f(ms - M);  // empty slot: weight 0, never read
+        w_s[s] = w;
+        if (w != 0.f) lloc += w * p.l[(size_t)(s0 + s) * n_h + h];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lloc += __shfl_xor_sync(0xffffffffu, lloc, o);
+    if (lane == 0) red[wid] = lloc;
+    __syncthreads();
     float Lsum = 0.f;
-    for (int s = s0; s < s1; ++s) {
-        float ms = p.m[(size_t)s * n_h + h];
-        if (ms != -INFINITY) Lsum += exp2f(ms - M) * p.l[(size_t)s * n_h + h];
-    }
+#pragma unroll
+    for (int i = 0; i < kCombineThreads / 32; ++i) Lsum += red[i];
     const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-    for (int c = threadIdx.x; c < d_c; c += blockDim.x) {
-        float acc = 0.f;
-        for (int s = s0; s < s1; ++s) {
-            float ms = p.m[(size_t)s * n_h + h];
-            if (ms != -INFINITY) acc += exp2f(ms - M) * p.o[((size_t)s * n_h + h) * d_c + c];
+    const size_t row_stride = (size_t)n_h * d_c;
+    const float *obase = p.o + ((size_t)s0 * n_h + h) * d_c;
+    float *dst = o_lat + ((size_t)r * n_h + h) * d_c;
+    if ((d_c & 3) == 0 && (reinterpret_cast<uintptr_t>(o_lat) & 15) == 0) {
+        for (int c4 = tid; c4 < d_c / 4; c4 += kCombineThreads) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int s = 0; s < S; ++s) {
+                const float w = w_s[s];
+                if (w == 0.f) continue;
+                const float4 v = reinterpret_cast<const float4 *>(obase + s * row_stride)[c4];
+                acc.x = fmaf(w, v.x, acc.x);
+                acc.y = fmaf(w, v.y, acc.y);
+                acc.z = fmaf(w, v.z, acc.z);
+                acc.w = fmaf(w, v.w, acc.w);
+            }
+            reinterpret_cast<float4 *>(dst)[c4] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
         }
-        o_lat[((size_t)r * n_h + h) * d_c + c] = acc * inv;
+    } else {
+        for (int c = tid; c < d_c; c += kCombineThreads) {
+            float acc = 0.f;
+            for (int s = 0; s < S; ++s) {
+                const float w = w_s[s];
+                if (w != 0.f) acc = fmaf(w, obase[s * row_stride + c], acc);
+            }
+            dst[c] = acc * inv;
+        }
     }
-    if (lse && threadIdx.x == 0)
+    if (lse && tid == 0)
         lse[(size_t)r * n_h + h] = Lsum > 0.f ? (M + log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
 }
 
@@ -254,7 +299,7 @@ cudaError_t launch_decode_simt(const mla_dims_t &d, int B, int s_q, const void *
 cudaError_t launch_combine(int rows, int n_h, int d_c, Partials p, const int32_t *seg_range,
                            int uniform, float *o_lat, float *lse, cudaStream_t st) {
     if (rows == 0) return cudaSuccess;
-    combine_kernel<<<dim3(rows, n_h), 128, 0, st>>>(n_h, d_c, p, seg_range, uniform, o_lat, lse);
+    combine_kernel<<<dim3(rows, n_h), kCombineThreads, 0, st>>>(n_h, d_c, p, seg_range, uniform, o_lat, lse);
     return cudaGetLastError();
 }
 

@@ -68,6 +68,13 @@ cudaError_t launch_absorb_q(const mla_dims_t &d, int T, const void *q_c, const v
 cudaError_t launch_out_proj(const mla_dims_t &d, int T, const float *o_lat, const void *w_uv,
                             void *o, mla_dtype_t out_dtype, cudaStream_t st);
 
+// Tensor-core projections (d_h = 128, d_c = 512, d_R = 64, bf16).
+bool proj_tc_supported(const mla_dims_t &d);
+cudaError_t launch_absorb_q_tc(const mla_dims_t &d, int T, const void *q_c, const void *q_r,
+                               const int32_t *pos, const void *w_uk, void *q_abs, cudaStream_t st);
+cudaError_t launch_out_proj_tc(const mla_dims_t &d, int T, const float *o_lat, const void *w_uv, void *o,
+                               mla_dtype_t out_dtype, cudaStream_t st);
+
 // CUDA-core split-KV decode.  Splits every query row into n_split segments of seg_len tokens.
 struct SimtPlan {
     int n_split;

@@ -99,9 +99,13 @@ out_proj_kernel(int T, int n_h, int d_h, int d_c, const float *__restrict__ o_la
 
 }  // namespace
 
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
 cudaError_t launch_absorb_q(const mla_dims_t &d, int T, const void *q_c, const void *q_r,
                             const int32_t *pos, const void *w_uk, void *q_abs, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
+    if (!(d.flags & MLA_FLAG_SIMT_PROJ) && proj_tc_supported(d) && aligned16(q_c) && aligned16(w_uk))
+        return launch_absorb_q_tc(d, T, q_c, q_r, pos, w_uk, q_abs, st);
     dim3 grid(d.n_h, (d.d_c + kAbsorbCols - 1) / kAbsorbCols, (T + kAbsorbTok - 1) / kAbsorbTok);
     size_t smem = sizeof(float) * kAbsorbTok * d.d_h;
     if (d.act_dtype == MLA_DTYPE_BF16) {
@@ -120,6 +124,8 @@ cudaError_t launch_absorb_q(const mla_dims_t &d, int T, const void *q_c, const v
 cudaError_t launch_out_proj(const mla_dims_t &d, int T, const float *o_lat, const void *w_uv,
                             void *o, mla_dtype_t out_dtype, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
+    if (!(d.flags & MLA_FLAG_SIMT_PROJ) && proj_tc_supported(d) && aligned16(o_lat) && aligned16(w_uv))
+        return launch_out_proj_tc(d, T, o_lat, w_uv, o, out_dtype, st);
     dim3 grid(d.n_h, (d.d_h + kOutRowsPerBlock - 1) / kOutRowsPerBlock, (T + kOutTok - 1) / kOutTok);
     dim3 block(kOutRowsPerBlock * 32);
     const bool wb = d.act_dtype == MLA_DTYPE_BF16;

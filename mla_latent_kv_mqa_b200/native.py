@@ -13,7 +13,8 @@ import os
 import re
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmla.so")
+# MLA_LIBRARY may point at another build of the same library (e.g. an instrumented one).
+LIB_PATH = os.environ.get("MLA_LIBRARY") or os.path.join(_PKG, "libmla.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "mla.h")
 
 if not os.path.exists(LIB_PATH):
@@ -35,6 +36,7 @@ MLA_DTYPE_F32 = 0
 MLA_DTYPE_BF16 = 1
 MLA_DTYPE_FP8_E4M3 = 2
 MLA_FLAG_SIMT_DECODE = 1
+MLA_FLAG_SIMT_PROJ = 2
 
 
 class MLAError(RuntimeError):

@@ -6,7 +6,8 @@ the plain 2e-2 bound; outputs of the log-normal-norm workload reach |o_lat| ~ 20
 rounding the absorbed query to bf16 alone (an fp64 emulation) already moves single elements
 by ~0.1, so the bound scales with the output's magnitude.  FP8
 content cache: relative L2 <= 3e-2 against the oracle run on its own dequantised cache
-(the same codes, checked bit-exact below); lse within 1e-2 absolute.  The fp32 toy layer
+(the same codes, checked bit-exact below); lse within 1e-2 * max(1, |lse|) (its bf16 error
+grows with the score magnitude: 0.018 on the log-normal workload's lse of 9..19).  The fp32 toy layer
 accumulates in fp32 over at most 256 tokens x 160 dims: relative L2 <= 1e-5.
 """
 import numpy as np
@@ -44,7 +45,7 @@ def _check(wl, got, ref, rows, heads, rel_tol, abs_tol):
     lse = lse.cpu().numpy()[rows][:, heads]
     e = dict(o_lat_rel=rel_l2(o_lat, ref.o_lat), o_rel=rel_l2(o, ref.o),
              o_lat_abs=scaled_max_abs(o_lat, ref.o_lat), o_abs=scaled_max_abs(o, ref.o),
-             lse_abs=max_abs(lse, ref.lse))
+             lse_abs=float(np.max(np.abs(lse - ref.lse) / np.maximum(1.0, np.abs(ref.lse)))))
     assert e["o_lat_rel"] <= rel_tol and e["o_rel"] <= rel_tol, e
     if abs_tol is not None:
         assert e["o_lat_abs"] <= abs_tol and e["o_abs"] <= abs_tol, e
@@ -70,7 +71,7 @@ SMALL = {
 def test_decode_matches_oracle_small(oracle_mod, case, simt):
     kw = dict(SMALL[case])
     wl = W.make_decode(name=case, **kw)
-    run = GpuRun(wl, flags=1 if simt else 0)
+    run = GpuRun(wl, flags=3 if simt else 0)  # 3: CUDA-core decode and projections
     run.fill_cache()
     got = run.step()
     rows, heads, ref = oracle_ref(wl, oracle_mod)
@@ -139,10 +140,15 @@ def test_append_bf16_scatter_is_bit_exact(oracle_mod):
         assert np.array_equal(bits[blk, slot, :d_c], _bf16_bits(wl.seq_c_kv(b)))
         # RoPE at position 0 is the identity: bit-exact
         assert np.array_equal(bits[blk[0], 0, d_c:], _bf16_bits(wl.seq_k_r(b)[0]))
-        # every other rotated key within half a bf16 ulp of the fp64 rotation
+        # every rotated key within one bf16 rounding (2^-9 relative) of the fp64 rotation, plus
+        # the fp32 rotation's own error, which scales with the pair (x_k, x_{k+d/2}) it mixes
         got = pool[blk, slot, d_c:].float().numpy()
-        want = np.stack([oracle_mod.rope(wl.seq_k_r(b)[p], float(p)) for p in range(L)])
-        assert np.all(np.abs(got - want) <= np.abs(want) * 2.0 ** -8 + 1e-30)
+        x = wl.seq_k_r(b).astype(np.float64)
+        want = np.stack([oracle_mod.rope(x[p], float(p)) for p in range(L)])
+        half = x.shape[1] // 2
+        pair = np.abs(x[:, :half]) + np.abs(x[:, half:])
+        pair = np.concatenate([pair, pair], 1)
+        assert np.all(np.abs(got - want) <= np.abs(want) * 2.0 ** -8 + pair * 2.0 ** -20)
     assert torch.isnan(pool[torch.from_numpy(~touched)].float()).all()
 
 
