@@ -27,8 +27,9 @@
  * Conventions shared by every call
  *   Memory     The caller owns every buffer; all pointers are device pointers of one
  *              device (the current device) unless a comment says otherwise.  The
- *              library allocates no device memory besides one static error word per
- *              device (see mla_get_last_device_error).
+ *              library allocates no device memory.  Its only device storage is static:
+ *              one error word per device (see mla_get_last_device_error) and the scratch
+ *              array of mla_decode_fixed_scratch.
  *   Streams    Calls only enqueue work on `stream` (NULL = the legacy default stream)
  *              and return; results are ready in stream order.
  *   Layouts    Row-major, contiguous, as each argument states.
@@ -158,6 +159,41 @@ mla_status_t mla_decode(const mla_dims_t *dims, int B, int s_q, const void *q_ab
                         const int32_t *block_table, int max_blocks_per_seq, int num_blocks,
                         const int32_t *seq_lens, int max_seq_len, void *workspace,
                         size_t workspace_bytes, float *o_lat, float *lse, mla_stream_t stream);
+
+/* ----------------------------------------------------------------------------------------
+ * mla_decode_fixed_scratch -- mla_decode without a caller workspace.  This call is a
+ * library convenience: the pages describe no counterpart to it.  It computes exactly what
+ * mla_decode computes, with the same arguments minus workspace / workspace_bytes.
+ *
+ * Who it is for: callers that cannot allocate device memory at decode time.  Examples are
+ * code running while a CUDA graph is being captured (an allocation there is either illegal
+ * or becomes part of the graph) and services with a fixed device-memory budget that is
+ * reserved up front.  Instead of a workspace argument, the call uses a scratch array of
+ * MLA_DECODE_FIXED_SCRATCH_BYTES that lives in the library's own static device storage.
+ * It allocates nothing itself.
+ *
+ *   Set-up     The first call on a device looks up that device's scratch address (the CUDA
+ *              runtime may load the library's device code at that moment).  Make the first
+ *              call on each device before any stream capture begins.  Later calls only read
+ *              a cached pointer.
+ *   Limit      If mla_decode_workspace_size(dims, B, s_q, max_seq_len) exceeds
+ *              MLA_DECODE_FIXED_SCRATCH_BYTES, the call returns MLA_ERR_WORKSPACE_TOO_SMALL
+ *              and launches nothing.  Use mla_decode with your own workspace instead.
+ *   Sharing    Every call on a device uses the same scratch array.  Calls whose executions
+ *              overlap on the device (on different streams without ordering between them)
+ *              race on it and produce wrong results.  Serialize them, for example on one
+ *              stream.  The scratch needs no clearing: every value the kernels read from it
+ *              is written earlier in the same call.
+ *   Errors     As for mla_decode; MLA_ERR_CUDA also when the scratch address cannot be
+ *              obtained.
+ * ---------------------------------------------------------------------------------------- */
+#define MLA_DECODE_FIXED_SCRATCH_BYTES (32u << 20) /* 32 MiB per device */
+mla_status_t mla_decode_fixed_scratch(const mla_dims_t *dims, int B, int s_q, const void *q_abs,
+                                      const void *kv_pool, const void *kr_pool,
+                                      const float *kv_scale, const int32_t *block_table,
+                                      int max_blocks_per_seq, int num_blocks,
+                                      const int32_t *seq_lens, int max_seq_len, float *o_lat,
+                                      float *lse, mla_stream_t stream);
 
 /* ----------------------------------------------------------------------------------------
  * mla_out_proj -- value up-projection after the aggregation (행렬 흡수 section):

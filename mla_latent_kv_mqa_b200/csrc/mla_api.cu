@@ -29,6 +29,30 @@ unsigned *device_error_word() {
     return g_err_addr[dev];
 }
 
+// Scratch of mla_decode_fixed_scratch: file-scope device storage, so that entry point never
+// allocates.  Every call on a device uses this one array.
+constexpr size_t kDecodeScratchBytes = (size_t)MLA_DECODE_FIXED_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_decode_scratch[kDecodeScratchBytes];
+
+namespace {
+void *g_scratch_addr[kMaxDevices] = {};
+std::mutex g_scratch_mu;
+}  // namespace
+
+// Device address of the scratch array on the current device.  The first call on a device
+// resolves it (and may load the module there); later calls return the cached pointer.
+void *decode_scratch() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress((void **)&p, g_decode_scratch) != cudaSuccess || !p) return nullptr;
+        g_scratch_addr[dev] = p;
+    }
+    return g_scratch_addr[dev];
+}
+
 }  // namespace mla
 
 using namespace mla;
@@ -157,6 +181,24 @@ mla_status_t mla_decode(const mla_dims_t *dims, int B, int s_q, const void *q_ab
     return from_cuda(launch_decode_simt(*dims, B, s_q, q_abs, kv_pool, kr_pool, kv_scale,
                                         block_table, max_blocks_per_seq, num_blocks, seq_lens,
                                         max_seq_len, workspace, o_lat, lse, st));
+}
+
+// mla_decode on the library's fixed scratch array instead of a caller workspace.  The size
+// check comes first; every other argument is checked by mla_decode itself.  The scratch holds
+// nothing between calls: the decode kernels write every workspace value before they read it.
+mla_status_t mla_decode_fixed_scratch(const mla_dims_t *dims, int B, int s_q, const void *q_abs,
+                                      const void *kv_pool, const void *kr_pool,
+                                      const float *kv_scale, const int32_t *block_table,
+                                      int max_blocks_per_seq, int num_blocks,
+                                      const int32_t *seq_lens, int max_seq_len, float *o_lat,
+                                      float *lse, mla_stream_t stream) {
+    void *scratch = decode_scratch();
+    if (!scratch) return MLA_ERR_CUDA;
+    if (mla_decode_workspace_size(dims, B, s_q, max_seq_len) > kDecodeScratchBytes)
+        return MLA_ERR_WORKSPACE_TOO_SMALL;
+    return mla_decode(dims, B, s_q, q_abs, kv_pool, kr_pool, kv_scale, block_table,
+                      max_blocks_per_seq, num_blocks, seq_lens, max_seq_len, scratch,
+                      kDecodeScratchBytes, o_lat, lse, stream);
 }
 
 mla_status_t mla_out_proj(const mla_dims_t *dims, int T, const float *o_lat, const void *w_uv,

@@ -64,12 +64,14 @@ _lib.mla_decode_workspace_size.argtypes = [_dp, _i, _i, _i]
 _lib.mla_decode_workspace_size.restype = _sz
 _lib.mla_decode.argtypes = [_dp, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _i, _vp, _sz, _vp,
                             _vp, _vp]
+_lib.mla_decode_fixed_scratch.argtypes = [_dp, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _i,
+                                          _vp, _vp, _vp]
 _lib.mla_out_proj.argtypes = [_dp, _i, _vp, _vp, _vp, _i, _vp]
 _lib.mla_get_last_device_error.argtypes = []
 _lib.mla_status_string.argtypes = [_i]
 _lib.mla_status_string.restype = ctypes.c_char_p
 _lib.mla_version.restype = _i
-for _f in ("mla_absorb_q", "mla_cache_append", "mla_decode", "mla_out_proj",
+for _f in ("mla_absorb_q", "mla_cache_append", "mla_decode", "mla_decode_fixed_scratch", "mla_out_proj",
            "mla_get_last_device_error"):
     getattr(_lib, _f).restype = _i
 
@@ -139,6 +141,17 @@ def mla_decode(dims, B, s_q, q_abs, kv_pool, kr_pool, kv_scale, block_table, max
                            _ptr(kv_scale), _ptr(block_table), max_blocks_per_seq, num_blocks,
                            _ptr(seq_lens), max_seq_len, _ptr(workspace), workspace_bytes,
                            _ptr(o_lat), _ptr(lse), _stream(stream)), "mla_decode")
+
+
+def mla_decode_fixed_scratch(dims, B, s_q, q_abs, kv_pool, kr_pool, kv_scale, block_table,
+                             max_blocks_per_seq, num_blocks, seq_lens, max_seq_len, o_lat, lse=None,
+                             stream=None):
+    """mla_decode on the library's static scratch array (no workspace argument)."""
+    _check(_lib.mla_decode_fixed_scratch(ctypes.byref(dims), B, s_q, _ptr(q_abs), _ptr(kv_pool),
+                                         _ptr(kr_pool), _ptr(kv_scale), _ptr(block_table),
+                                         max_blocks_per_seq, num_blocks, _ptr(seq_lens), max_seq_len,
+                                         _ptr(o_lat), _ptr(lse), _stream(stream)),
+           "mla_decode_fixed_scratch")
 
 
 def mla_out_proj(dims, T, o_lat, w_uv, o, out_dtype=MLA_DTYPE_F32, stream=None):
