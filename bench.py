@@ -272,6 +272,12 @@ def run_mine(args):
             g_dec.replay()
             g_e2e.replay()
         stream.synchronize()
+        # let the SM clock ramp up under sustained load before timing (idle boards sit far below boost)
+        t_end = time.time() + args.clock_warmup_s
+        while time.time() < t_end:
+            for _ in range(20):
+                g_step.replay()
+            stream.synchronize()
 
         K = args.steps
         mk = lambda: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
@@ -359,8 +365,9 @@ def run_mine(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--clock-warmup-s", type=float, default=1.5)
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
     ap.add_argument("--config", default="v3", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")

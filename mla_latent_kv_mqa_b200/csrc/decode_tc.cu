@@ -325,7 +325,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv5, const __grid_consta
     cluster_sync();
     const uint32_t tmem = ctrl->tmem_base;
     const uint32_t peer = rank ^ 1u;
-    if (threadIdx.x == 0) TRACE(20 + rank, 0);
+    if (threadIdx.x == 0) TRACE(20 + rank, (uint32_t)clock64() >> 8);
     auto fail = [&]() {
         if (*abort_flag == 0) {
             *abort_flag = 1;
@@ -754,7 +754,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv5, const __grid_consta
 
     // ---- teardown: both CTAs quiesce before either releases TMEM or exits ----
     __syncwarp();
-    if (threadIdx.x == 0) TRACE(22 + rank, 0);
+    if (threadIdx.x == 0) TRACE(22 + rank, (uint32_t)clock64() >> 8);
     tc_fence_before();
     __syncthreads();
     cluster_sync();
