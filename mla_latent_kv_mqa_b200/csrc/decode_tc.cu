@@ -9,19 +9,25 @@
 //     S[128 x 64]  = Q[128 x 576] . KV[64 x 576]^T      (QK, K = 576)
 //     O[128 x 512] += P[128 x 64] . V[64 x 512]         (PV, V = the c_j part of KV)
 //
-// Decomposition.  O in fp32 is 128 lanes x 512 columns: all of one SM's tensor memory.  A
-// 2-CTA cluster therefore splits the two contractions between two SMs instead of splitting
-// either one:
-//   CTA 0 ("QK"): Q (576 bf16 per head) lives in TMEM columns [0,288); three S buffers of 64
-//     columns follow.  A TMA warp streams each page's 576-wide rows (9 column blocks of 64,
-//     128-byte swizzle) into a 3-stage ring; one thread issues 36 tcgen05.mma (M=128, N=64,
-//     K=16, A from TMEM); 4 softmax warps (one head per thread) run the online softmax in fp32
-//     and ship bf16 P (16 KB) plus per-head rescale factors to CTA 1 with st.async.
-//   CTA 1 ("PV"): O lives in all 512 TMEM columns.  A TMA warp streams the same page's 512
-//     content columns (mostly L2 hits) into a 2-stage ring; one thread issues 8 tcgen05.mma
-//     (M=128, N=256, K=16, A = P, B = V read MN-major); 4 warps zero the rows of ragged last
-//     pages, apply the (rare) lazy rescale of O rows, release P slots and write each segment's
-//     partial O.
+// Decomposition.  O in fp32 is 128 lanes x 512 columns: all of one SM's tensor memory, so a
+// 2-CTA cluster splits the two contractions between two SMs:
+//   CTA 0 ("QK"): Q (576 bf16 per head, 288 TMEM columns) sits in TMEM next to three 64-column
+//     S buffers.  One TMA thread streams whole pages (one 72 KB 3-D box each) into a 3-stage
+//     ring; the segment's Q arrives through the same ring.  Two MMA threads split each page's
+//     36 tcgen05.mma (M = 128, N = 64, K = 16, A from TMEM) by column blocks (one thread cannot
+//     issue N = 64 MMAs as fast as the tensor core runs them).  Eight softmax warps, two per TMEM lane quarter and each
+//     owning 32 of a page's 64 columns, run the online softmax in fp32 and put bf16 P into 32
+//     spare TMEM columns.  Four sender warps take it from there and store P, per-head rescale
+//     factors and a flag into CTA 1's shared memory with st.async.  The distributed-shared-
+//     memory link (about 20 GB/s per SM pair) is the slowest step of the page, so the softmax
+//     warps hand off and go on to the next page while the senders drain it, and the TMA
+//     engine stays free for the page stream.
+//   CTA 1 ("PV"): O lives in all 512 TMEM columns.  A TMA thread streams the same page's 512
+//     content columns (mostly L2 hits) as two 32 KB halves into a 4-deep ring; one thread
+//     issues 8 tcgen05.mma per page (M = 128, N = 256, K = 16, A = P, B = V read MN-major)
+//     and, through a multicast commit, hands the P slot back to CTA 0 the moment those MMAs
+//     are done.  Four warps zero the rows of ragged last pages, apply the (rare) lazy
+//     rescale of O rows, and write each segment's partial O with coalesced stores.
 // QK : PV work is 576 : 512, so the two tensor pipes are nearly balanced and no FLOP or byte
 // is done twice (the second read of a page is an L2 hit).
 //
@@ -32,8 +38,9 @@
 // Lazy rescaling (log2 units): a row's running max only moves when a page's max exceeds it by
 // more than 8, so P stays <= 256 and O rows are rescaled only on those (rare) pages.
 //
-// Every mbarrier wait is bounded (2 s); on give-up a CTA raises an abort flag in itself and its
-// peer, records MLA_ERR_DEVICE_TIMEOUT and leaves through the normal teardown.
+// Every wait is bounded (2 s).  On give-up a CTA raises an abort flag in itself and its peer
+// and records MLA_ERR_DEVICE_TIMEOUT; before the teardown every thread that started copies or
+// MMAs waits (again bounded) for them, so no asynchronous write targets a CTA that has left.
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -47,66 +54,68 @@ namespace {
 using namespace sm100;
 
 constexpr int NH = 128, DC = 512, ROW = 576, PG = 64;
-constexpr int CB = PG * 128;                // one 64-row x 64-column bf16 box, 128-byte swizzle
+constexpr int CB = PG * 128;                // one 64-row x 64-column bf16 tile, 128-byte swizzle
 constexpr int NCB = ROW / 64;               // 9 column blocks per cache row
-// ---- QK CTA shared memory ----
-// A page (64 tokens x 576) is one TMA operation (a 3-D box {64, 64, 9} over the cache viewed as
-// column blocks), so one issuing thread streams whole pages: TMA operations of one thread are
-// served one after another, and 8 KB operations would cap a thread at ~24 GB/s.
-constexpr int KV_STAGES = 2;
+// ---- QK CTA shared memory: a ring of whole pages ----
+// A page (64 tokens x 576) is one TMA operation: a 3-D box {64, 64, 9} over the cache viewed as
+// column blocks, landing as 9 K-major SW128 tiles.  A segment's Q (128 heads x 576) takes two
+// ring stages (heads 0-63, 64-127) through the same box shape over q_abs.
+constexpr int KV_STAGES = 3;
 constexpr int KV_STAGE = NCB * CB;          // 73728
-constexpr int QC_BYTES = 8 * CB;            // Q content of 64 heads (8 column blocks): 65536
-constexpr int QROPE_OFF = KV_STAGES * KV_STAGE;  // 147456: Q RoPE part, [128 heads x 64] bf16
-constexpr int STAGE_OFF = QROPE_OFF + 2 * CB;
+constexpr int DATA_A = KV_STAGES * KV_STAGE;
+// ---- PV CTA shared memory ----
+constexpr int VH_STAGES = 4;                // ring of half pages: 4 column blocks (256 columns)
+constexpr int VH_STAGE = 4 * CB;            // 32768
+constexpr int V_OFF = 0;
+constexpr int P_OFF = VH_STAGES * VH_STAGE;
 constexpr int P_TILE = NH * PG * 2;         // 16384: P[128 heads][64 tokens] bf16, SW128 K-major
 constexpr int P_FACT = P_TILE;              // 128 fp32 rescale factors
-constexpr int P_FLAG = P_TILE + NH * 4;     // one u32: any factor != 1
-constexpr int P_SLOT = 17408;               // message slot, padded to 1 KB
-constexpr uint32_t MSG_BYTES = P_TILE + NH * 4 + 16;  // bulk-copy size (multiple of 16)
-constexpr int STAGE_SLOTS = 2;              // local P staging slots
-constexpr int DATA_A = STAGE_OFF + STAGE_SLOTS * P_SLOT;
-// ---- PV CTA shared memory ----
-constexpr int V_STAGES = 2;
-constexpr int V_STAGE = (DC / 64) * CB;     // 65536: the content columns of one page
-constexpr int V_OFF = 0;
-constexpr int P_OFF = V_STAGES * V_STAGE;
-constexpr int P_SLOTS = 3;                  // P receive slots
-constexpr int EPI_OFF = P_OFF + P_SLOTS * P_SLOT;  // 2 x 16 KB staging of O chunks for TMA stores
-constexpr int EPI_CHUNK = NH * 128;         // [128 heads x 32 fp32] with 128-byte swizzle
-constexpr int DATA_B = EPI_OFF + 2 * EPI_CHUNK;
+constexpr int P_FLAG = P_TILE + NH * 4;     // one u32: some factor != 1
+constexpr uint32_t MSG_BYTES = P_TILE + NH * 4 + 4;  // bytes st.async delivers per page
+constexpr int P_SLOT = 17408;               // slot stride, 1 KB aligned
+constexpr int P_SLOTS = 3;
+constexpr int DATA_B = P_OFF + P_SLOTS * P_SLOT;
 constexpr int DATA = DATA_A > DATA_B ? DATA_A : DATA_B;
-static_assert(P_SLOT % 1024 == 0 && P_OFF % 1024 == 0 && STAGE_OFF % 1024 == 0 &&
-              QROPE_OFF % 1024 == 0 && EPI_OFF % 1024 == 0, "swizzled tiles need 1 KB alignment");
+static_assert(P_SLOT % 1024 == 0 && P_OFF % 1024 == 0 && VH_STAGE % 1024 == 0,
+              "swizzled tiles need 1 KB alignment");
 static_assert(MSG_BYTES <= (uint32_t)P_SLOT, "message slot");
-// ---- QK CTA tensor memory: Q content, then 2 sets x 2 partial S accumulators ----
+// ---- QK CTA tensor memory: three S buffers, then Q (content and RoPE part) ----
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t Q_COL = 0, S_COL = DC / 2;  // 256
-constexpr int S_SETS = 2;
-static_assert(S_COL + S_SETS * 2 * PG <= TMEM_COLS, "QK-CTA TMEM budget");
-// The 36 k-steps of QK are split between two issuing warps (one issuer cannot keep the
-// tensor pipe busy at N = 64): warp 1 takes column blocks 0..4, warp 2 blocks 5..8 (block 8
-// is the RoPE part, with A read from shared memory).
-constexpr int SPLIT_CB = 5;
-constexpr int THREADS = 256;                // 8 warps
-// Each stage is filled by two producer warps (warp 0: column blocks 0..4, warp 7: 5..8; PV CTA:
-// 0..3 and 4..7), i.e. two TMA streams that the copy engine serves in parallel.
-constexpr int PROD2_WARP = 7;
-constexpr int SPLIT_LOAD = 5;
-constexpr int SM_THREAD0 = 96;              // first softmax thread (warps 3..6)
+constexpr int S_SETS = 3;
+constexpr uint32_t S_COL = 0;
+constexpr uint32_t Q_COL = S_SETS * PG;     // 192; column block c of Q at Q_COL + 32 c
+constexpr uint32_t P_COL = Q_COL + NCB * 32;  // 480: P of one page, bf16 pairs (32 columns)
+static_assert(P_COL + PG / 2 <= TMEM_COLS, "QK-CTA TMEM budget");
+// ---- threads ----
+constexpr int THREADS = 480;                // 15 warps
+constexpr int SM_WARP0 = 3;                 // QK CTA: softmax warps 3..10
+constexpr int SM_THREADS = 256;
+constexpr int SD_WARP0 = 11;                // QK CTA: sender warps 11..14 (P -> CTA 1 by st.async)
+constexpr int SD_THREADS = 128;
+constexpr int EP_WARP0 = 2;                 // PV CTA: correction / epilogue warps 2..5
 constexpr float RESCALE_LOG2 = 8.0f;
 
 struct __align__(8) Ctrl {
+    // QK CTA
     uint64_t kv_full[KV_STAGES], kv_empty[KV_STAGES];
     uint64_t s_full[S_SETS], s_free[S_SETS];
-    uint64_t q_ready, rope_full, rope_free;
-    uint64_t pfree[P_SLOTS];
-    uint64_t v_full[V_STAGES], v_empty[V_STAGES], v_ready[V_STAGES];
+    uint64_t k0_done[S_SETS];   // MMA thread 0 has issued its part of the page in this S buffer
+    uint64_t q_ready;
+    uint64_t p_ready, p_taken;  // P in TMEM: written by the softmax / read by the senders
+    uint64_t pfree[P_SLOTS];    // P slot of CTA 1 reusable: its PV MMAs done (1) + read by 4 warps
+    // PV CTA
+    uint64_t v_full[VH_STAGES], v_empty[VH_STAGES], v_ready[VH_STAGES];
     uint64_t p_full[P_SLOTS], pv_done[P_SLOTS];
     uint64_t corr_done, o_free;
+    uint64_t mma_idle[2];       // drains: one per MMA-issuing thread
     uint32_t tmem_base;
     uint32_t abort;
+    uint32_t never;             // stays 0: the abort word of drain waits, which must not give up early
+    float lx[2][NH];            // QK CTA: the second softmax half's row sums, by segment parity
+    float fac[2][NH];           // QK CTA: per-head rescale factors of a page, by page parity
 };
 constexpr int SMEM_BYTES = 1024 + DATA + (int)((sizeof(Ctrl) + 127) / 128 * 128);
+static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 
 struct Params {
     const int32_t *bt;
@@ -114,7 +123,8 @@ struct Params {
     const int32_t *seq_lens;
     int s_q, rows, max_seq_len;
     const int32_t *work;  // [pairs][4]: first row, first page, number of pages
-    float *o_part, *m_part, *l_part;
+    uint32_t *o_part;  // [slot][d_c / 2][n_h]: bf16 pairs of columns (c = 2k, 2k + 1) per head
+    float *m_part, *l_part;
     float scale_log2;
     unsigned *err;
 };
@@ -196,9 +206,6 @@ __device__ __forceinline__ void st_shared_v4(uint32_t a, uint32_t x, uint32_t y,
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w)
                  : "memory");
 }
-__device__ __forceinline__ void st_shared_u32(uint32_t a, uint32_t x) {
-    asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(x) : "memory");
-}
 __device__ __forceinline__ void named_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
@@ -212,48 +219,33 @@ __device__ __forceinline__ bool named_red_or(bool v, int id, int n) {
         : "memory");
     return r != 0;
 }
-__device__ __forceinline__ bool named_red_and(bool v, int id, int n) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-        "barrier.cta.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)v), "r"(id), "r"(n)
-        : "memory");
-    return r != 0;
-}
 // 2^x on the SFU (ex2.approx, flush-to-zero): P only needs bf16 precision.
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
-// Bulk copy of `bytes` from this CTA's shared memory to another CTA's (TMA engine), completing
-// `bytes` on the destination's mbarrier.
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_remote, uint32_t src_local, uint32_t bytes,
-                                                  uint32_t bar_remote) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            dst_remote),
-        "r"(src_local), "r"(bytes), "r"(bar_remote)
-        : "memory");
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+__device__ __forceinline__ float max32(const float (&x)[32]) {
+    float a = fmaxf(x[0], x[1]), b = fmaxf(x[2], x[3]), c = fmaxf(x[4], x[5]), d = fmaxf(x[6], x[7]);
+#pragma unroll
+    for (int j = 8; j < 32; j += 8) {
+        a = fmaxf(a, fmaxf(x[j + 0], x[j + 1]));
+        b = fmaxf(b, fmaxf(x[j + 2], x[j + 3]));
+        c = fmaxf(c, fmaxf(x[j + 4], x[j + 5]));
+        d = fmaxf(d, fmaxf(x[j + 6], x[j + 7]));
+    }
+    return fmaxf(fmaxf(a, b), fmaxf(c, d));
 }
-__device__ __forceinline__ void bulk_wait_read_le1() {
-    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 #ifdef MLA_TRACE
 // Development instrumentation: globaltimer stamps of pipeline events of one cluster.  Each warp
 // of each CTA writes its own 4096-entry region (no atomics on the traced path).
-constexpr int kTraceMax = 1 << 16;
 constexpr int kTraceRegion = 4096;
+constexpr int kTraceMax = 2 * 16 * kTraceRegion;
 __device__ uint32_t g_trace[2 * kTraceMax];
-__device__ uint32_t g_trace_n;
 __device__ __forceinline__ void trace_event(int pair, uint32_t code, uint32_t unit, uint32_t &n) {
     if (pair != MLA_TRACE) return;
-    const uint32_t region = cluster_ctarank() * 8 + (threadIdx.x >> 5);
+    const uint32_t region = cluster_ctarank() * 16 + (threadIdx.x >> 5);
     if (n < kTraceRegion) {
         const uint32_t i = region * kTraceRegion + n++;
         g_trace[2 * i] = code | (unit << 8);
@@ -265,13 +257,28 @@ __device__ __forceinline__ void trace_event(int pair, uint32_t code, uint32_t un
 #define TRACE(code, unit) ((void)0)
 #endif
 
-// Named barriers of the 4 softmax warps (QK CTA) and of the 4 epilogue warps (PV CTA).
-constexpr int BAR_Q = 1, BAR_FLAG = 2, BAR_OK = 3, BAR_EPI = 4;
+#ifdef MLA_PROF
+// Development instrumentation: per role and phase, clock cycles summed over a warp's pages
+// (lane 0), added once per warp into g_prof[rank][warp][phase] at the end; [..][..][7] counts pages.
+__device__ unsigned long long g_prof[2][16][8];
+#define PROF_DECL long long pf_acc[8] = {}; long long pf_t = clock64();
+#define PROF_MARK(i) do { const long long _n = clock64(); pf_acc[i] += _n - pf_t; pf_t = _n; } while (0)
+#define PROF_PAGE() (pf_acc[7] += 1)
+#define PROF_FLUSH() do { if (lane == 0) for (int _i = 0; _i < 8; ++_i) \
+    atomicAdd(&g_prof[cluster_ctarank()][warp][_i], (unsigned long long)pf_acc[_i]); } while (0)
+#else
+#define PROF_DECL
+#define PROF_MARK(i) ((void)0)
+#define PROF_PAGE() ((void)0)
+#define PROF_FLUSH() ((void)0)
+#endif
+
+// Named barriers: the 256 softmax threads and the 128 sender threads (QK CTA).
+constexpr int BAR_FAIL = 1, BAR_Q = 2, BAR_SFAIL = 3, BAR_SFLAG = 4;
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
-decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv5, const __grid_constant__ CUtensorMap tm_kv4,
-                 const __grid_constant__ CUtensorMap tm_q4, const __grid_constant__ CUtensorMap tm_qr,
-                 const __grid_constant__ CUtensorMap tm_o, const Params P) {
+decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_constant__ CUtensorMap tm_kv4,
+                 const __grid_constant__ CUtensorMap tm_q9, const Params P) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_u32(smem_raw);
     const uint32_t data_s = (raw_s + 1023u) & ~1023u;
@@ -288,29 +295,33 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv5, const __grid_consta
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < KV_STAGES; ++i) {
-            mbar_init(bar(ctrl->kv_full[i]), 2);    // two producer warps
-            mbar_init(bar(ctrl->kv_empty[i]), 2);  // both QK issuers (or the Q copy) release a stage
+            mbar_init(bar(ctrl->kv_full[i]), 1);
+            mbar_init(bar(ctrl->kv_empty[i]), 2);  // both MMA threads (or the Q copy, twice)
         }
         for (int i = 0; i < S_SETS; ++i) {
             mbar_init(bar(ctrl->s_full[i]), 2);
-            mbar_init(bar(ctrl->s_free[i]), 4);
+            mbar_init(bar(ctrl->k0_done[i]), 1);
+            mbar_init(bar(ctrl->s_free[i]), SM_THREADS / 32);
         }
         mbar_init(bar(ctrl->q_ready), 1);
-        mbar_init(bar(ctrl->rope_full), 1);
-        mbar_init(bar(ctrl->rope_free), 1);
+        mbar_init(bar(ctrl->p_ready), SM_THREADS / 32);
+        mbar_init(bar(ctrl->p_taken), SD_THREADS / 32);
         for (int i = 0; i < P_SLOTS; ++i) {
-            mbar_init(bar(ctrl->pfree[i]), 1);
+            mbar_init(bar(ctrl->pfree[i]), 1 + 4);
             mbar_init(bar(ctrl->p_full[i]), 1);
             mbar_init(bar(ctrl->pv_done[i]), 1);
         }
-        for (int i = 0; i < V_STAGES; ++i) {
-            mbar_init(bar(ctrl->v_full[i]), 2);     // two producer warps
+        for (int i = 0; i < VH_STAGES; ++i) {
+            mbar_init(bar(ctrl->v_full[i]), 1);
             mbar_init(bar(ctrl->v_empty[i]), 1);
             mbar_init(bar(ctrl->v_ready[i]), 4);
         }
         mbar_init(bar(ctrl->corr_done), 4);
         mbar_init(bar(ctrl->o_free), 4);
+        mbar_init(bar(ctrl->mma_idle[0]), 1);
+        mbar_init(bar(ctrl->mma_idle[1]), 1);
         ctrl->abort = 0;
+        ctrl->never = 0;
         if (rank == 1)
             for (int i = 0; i < P_SLOTS; ++i) mbar_arrive_expect_tx(bar(ctrl->p_full[i]), MSG_BYTES);
         fence_mbarrier_init_cluster();
@@ -323,6 +334,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv5, const __grid_consta
     __syncthreads();
     tc_fence_after();
     cluster_sync();
+    // Everything above overlaps the scheduler kernel; its work list is read from here on.
+    pdl_trigger();
+    pdl_wait();
     const uint32_t tmem = ctrl->tmem_base;
     const uint32_t peer = rank ^ 1u;
     if (threadIdx.x == 0) TRACE(20 + rank, (uint32_t)clock64() >> 8);
@@ -333,90 +347,103 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv5, const __grid_consta
             record_error(P.err, kErrTimeout);
         }
     };
+    // Drain waits ignore the abort flag: they wait for hardware that is already running.
+    volatile uint32_t *never = &ctrl->never;
 
     if (rank == 0) {
         // ===================================== QK CTA =====================================
-        if ((warp == 0 || warp == PROD2_WARP) && lane == 0) {  // TMA producers (two streams)
-            const int half = warp == 0 ? 0 : 1;
-            prefetch_tensormap(half ? &tm_kv4 : &tm_kv5);
-            prefetch_tensormap(&tm_q4);
-            if (!half) prefetch_tensormap(&tm_qr);
+        if (warp == 0 && lane == 0) {  // TMA producer: per segment 2 Q stages, then its pages
+            prefetch_tensormap(&tm_kv9);
+            prefetch_tensormap(&tm_q9);
             PageIt it;
             it.init(P, pair);
             Ring st{0, 0};
-            uint32_t nseg = 0;
+            int issued[KV_STAGES];           // phase + 1 of the last copy into each stage (0: none)
+            for (int i = 0; i < KV_STAGES; ++i) issued[i] = 0;
+            uint32_t nph[KV_STAGES] = {};
             int u = 0;
             bool ok = true;
+            PROF_DECL
+            auto load = [&](const CUtensorMap *map, int y) -> bool {
+                if (!wait(bar(ctrl->kv_empty[st.i]), st.ph ^ 1u, abort_flag)) return false;
+                PROF_MARK(0);
+                mbar_arrive_expect_tx(bar(ctrl->kv_full[st.i]), KV_STAGE);
+                tma_load_3d(data_s + st.i * KV_STAGE, map, 0, y, 0, bar(ctrl->kv_full[st.i]));
+                PROF_MARK(1);
+                issued[st.i] = 1;
+                nph[st.i] = st.ph;
+                st.adv(KV_STAGES);
+                return true;
+            };
             while (ok && !it.done()) {
                 if (it.first) {
-                    if (!half) {
-                        if (!(ok = wait(bar(ctrl->rope_free), (nseg & 1u) ^ 1u, abort_flag))) break;
-                        mbar_arrive_expect_tx(bar(ctrl->rope_full), 2 * CB);
-                        tma_load_2d(data_s + QROPE_OFF, &tm_qr, DC, it.r * NH, bar(ctrl->rope_full));
-                    }
-                    // Q content: stage s <- heads 0-63, stage s+1 <- heads 64-127; this stream
-                    // loads column blocks 4*half .. 4*half+3 of each
-                    for (int hh = 0; hh < 2 && ok; ++hh) {
-                        if (!(ok = wait(bar(ctrl->kv_empty[st.i]), st.ph ^ 1u, abort_flag))) break;
-                        mbar_arrive_expect_tx(bar(ctrl->kv_full[st.i]), QC_BYTES / 2);
-                        tma_load_3d(data_s + st.i * KV_STAGE + half * 4 * CB, &tm_q4, 0, it.r * NH + hh * 64,
-                                    half * 4, bar(ctrl->kv_full[st.i]));
-                        st.adv(KV_STAGES);
-                    }
-                    if (!ok) break;
-                    ++nseg;
-                    if (!half) TRACE(1, u);
+                    if (!(ok = load(&tm_q9, it.r * NH) && load(&tm_q9, it.r * NH + 64))) break;
+                    TRACE(1, u);
                 }
-                if (!(ok = wait(bar(ctrl->kv_empty[st.i]), st.ph ^ 1u, abort_flag))) break;
-                const int blk = block_of(P, it.r, it.pg);
-                const int cbs = half ? NCB - SPLIT_LOAD : SPLIT_LOAD;
-                mbar_arrive_expect_tx(bar(ctrl->kv_full[st.i]), cbs * CB);
-                tma_load_3d(data_s + st.i * KV_STAGE + half * SPLIT_LOAD * CB, half ? &tm_kv4 : &tm_kv5, 0,
-                            blk * PG, half * SPLIT_LOAD, bar(ctrl->kv_full[st.i]));
-                st.adv(KV_STAGES);
-                if (!half) TRACE(2, u);
+                if (!(ok = load(&tm_kv9, block_of(P, it.r, it.pg) * PG))) break;
+                PROF_PAGE();
+                TRACE(2, u);
                 ++u;
                 it.next(P);
             }
             if (!ok) fail();
-        } else if ((warp == 1 || warp == 2) && lane == 0) {  // MMA issuers: partial S = Q . KV^T
+            PROF_FLUSH();
+            for (int i = 0; i < KV_STAGES; ++i)  // drain: every copy this thread started has landed
+                if (issued[i]) wait(bar(ctrl->kv_full[i]), nph[i], never);
+        } else if ((warp == 1 || warp == 2) && lane == 0) {  // MMA issuers: S += Q . KV^T, split K
+            // Both threads work on every page: thread 0 column blocks 0-4, thread 1 blocks 5-8 (the
+            // RoPE part).  One thread cannot issue N = 64 MMAs as fast as the tensor core runs them,
+            // and splitting the page (not alternating pages) keeps each stage busy for the shortest
+            // time.  All MMAs accumulate: the softmax zeroes an S buffer when it has read it.
+            // Thread 1 issues a page's part only after thread 0 has issued its own (k0_done, with
+            // the tcgen05 thread-sync fences on both sides), so every page sums in the same order
+            // and results are bitwise reproducible; thread 0 meanwhile goes on to the next page.
             constexpr uint32_t idesc = idesc_bf16(128, PG, false, false);
-            const int part = warp - 1;                  // 0: blocks 0..4, 1: blocks 5..8
-            const int cb0 = part ? SPLIT_CB : 0, cb1 = part ? NCB : SPLIT_CB;
+            const int part = warp - 1;
+            const int cb0 = part ? 5 : 0, cb1 = part ? NCB : 5;
             PageIt it;
             it.init(P, pair);
             Ring st{0, 0}, sb{0, 0};
             uint32_t qn = 0;
             int u = 0;
-            bool ok = true;
+            bool ok = true, any = false;
+            PROF_DECL
             while (ok && !it.done()) {
                 if (it.first) {
                     st.adv(KV_STAGES, 2);  // the segment's Q stages (copied to TMEM by the softmax warps)
+                    PROF_MARK(4);
                     if (!(ok = wait(bar(ctrl->q_ready), qn & 1u, abort_flag))) break;
-                    if (part && !(ok = wait(bar(ctrl->rope_full), qn & 1u, abort_flag))) break;
+                    PROF_MARK(0);
                     ++qn;
                 }
+                PROF_MARK(4);
                 if (!(ok = wait(bar(ctrl->s_free[sb.i]), sb.ph ^ 1u, abort_flag))) break;
-                tc_fence_after();  // orders our S writes after the softmax's TMEM reads
+                if (part && !(ok = wait(bar(ctrl->k0_done[sb.i]), sb.ph, abort_flag))) break;
+                PROF_MARK(1);
+                tc_fence_after();  // orders the MMAs after the softmax's TMEM zeroing / thread 0's MMAs
                 // TMA-filled shared memory needs no tcgen05 fence: the mbarrier completion already
-                // makes it visible to the MMAs issued after the wait.
+                // makes it visible to MMAs issued after the wait.
                 if (!(ok = wait(bar(ctrl->kv_full[st.i]), st.ph, abort_flag))) break;
-                const uint32_t d = tmem + S_COL + sb.i * 2 * PG + part * PG;
+                PROF_MARK(2);
+                TRACE(6 + part, u);
+                const uint32_t d = tmem + S_COL + sb.i * PG;
                 const uint32_t kvb = data_s + st.i * KV_STAGE;
+#pragma unroll 1
                 for (int cb = cb0; cb < cb1; ++cb) {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint64_t b = sdesc_sw128(kvb + cb * CB + k * 32, 16, 1024);
-                        const uint32_t acc = (cb == cb0 && k == 0) ? 0u : 1u;
-                        if (cb < NCB - 1)
-                            mma_ts(d, tmem + Q_COL + (cb * 4 + k) * 8, b, idesc, acc);
-                        else
-                            mma_ss(d, sdesc_sw128(data_s + QROPE_OFF + k * 32, 16, 1024), b, idesc, acc);
-                    }
+                    for (int k = 0; k < 4; ++k)
+                        mma_ts(d, tmem + Q_COL + (cb * 4 + k) * 8, sdesc_sw128(kvb + cb * CB + k * 32, 16, 1024),
+                               idesc, 1u);
+                }
+                if (!part) {
+                    tc_fence_before();
+                    mbar_arrive(bar(ctrl->k0_done[sb.i]));
                 }
                 mma_commit(bar(ctrl->kv_empty[st.i]));
                 mma_commit(bar(ctrl->s_full[sb.i]));
-                if (part && it.last()) mma_commit(bar(ctrl->rope_free));
+                PROF_MARK(3);
+                PROF_PAGE();
+                any = true;
                 TRACE(3 + part, u);
                 ++u;
                 st.adv(KV_STAGES);
@@ -424,36 +451,39 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv5, const __grid_consta
                 it.next(P);
             }
             if (!ok) fail();
-        } else if (warp >= 3 && warp <= 6) {  // softmax warps: thread = head
-            const int t = threadIdx.x - SM_THREAD0;
-            const int sub = warp & 3;
-            const int h = sub * 32 + lane;
-            const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
-            uint32_t p_slot_r[P_SLOTS], p_full_r[P_SLOTS];
-            for (int i = 0; i < P_SLOTS; ++i) {
-                p_slot_r[i] = mapa(data_s + P_OFF + i * P_SLOT, 1);
-                p_full_r[i] = mapa(bar(ctrl->p_full[i]), 1);
+            PROF_FLUSH();
+            if (any) {  // drain: the MMAs this thread issued are complete before TMEM is released
+                mma_commit(bar(ctrl->mma_idle[part]));
+                wait(bar(ctrl->mma_idle[part]), 0u, never);
             }
+        } else if (warp >= SM_WARP0 && warp < SM_WARP0 + 8) {  // softmax: 2 warps per lane quarter
+            const int t = threadIdx.x - SM_WARP0 * 32;          // 0..255
+            const int quarter = warp & 3;
+            const int half = (warp - SM_WARP0) >> 2;            // which 32 of the 64 columns
+            const int h = quarter * 32 + lane;                  // head = TMEM lane
+            const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
             PageIt it;
             it.init(P, pair);
-            Ring st{0, 0}, sb{0, 0}, ps{0, 0}, sg{0, 0};  // sg: local P staging slot
+            Ring st{0, 0}, sb{0, 0};
             float m_used = -INFINITY, l = 0.f;
-            int u = 0;
-            bool ok = true, pfail = false;  // pfail: thread 0 gave up waiting for a P slot
+            int u = 0, seg = 0;
+            bool ok = true;
 
-            // Q content of a segment (2 stages: heads 0-63, 64-127) -> this thread's TMEM lane.
+            // Q of a segment (2 stages: heads 0-63, 64-127) -> TMEM lane h; this half copies
+            // column blocks 0-4 (half 0) or 5-8 (half 1).  Uniform across the 256 threads.
             auto load_q = [&]() -> bool {
                 const Ring q0 = st;
                 st.adv(KV_STAGES);
                 const Ring q1 = st;
                 st.adv(KV_STAGES);
-                bool w = wait(bar(ctrl->kv_full[q0.i]), q0.ph, abort_flag) &&
-                         wait(bar(ctrl->kv_full[q1.i]), q1.ph, abort_flag);
-                if (!named_red_and(w, BAR_OK, 128)) return false;
+                const bool w = wait(bar(ctrl->kv_full[q0.i]), q0.ph, abort_flag) &&
+                               wait(bar(ctrl->kv_full[q1.i]), q1.ph, abort_flag);
+                if (named_red_or(!w, BAR_Q, SM_THREADS)) return false;
                 const int rr = h & 63;
                 const uint32_t rowa = data_s + ((h >> 6) ? q1.i : q0.i) * KV_STAGE + rr * 128;
+                const int cb0 = half ? 5 : 0, cb1 = half ? NCB : 5;
 #pragma unroll 1
-                for (int cb = 0; cb < 8; ++cb) {
+                for (int cb = cb0; cb < cb1; ++cb) {
                     uint32_t v[32];
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
@@ -467,7 +497,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv5, const __grid_consta
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                named_sync(BAR_Q, 128);
+                named_sync(BAR_Q, SM_THREADS);
                 if (t == 0) {
                     for (int k = 0; k < 2; ++k) {
                         mbar_arrive(bar(ctrl->kv_empty[q0.i]));
@@ -478,147 +508,242 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv5, const __grid_consta
                 return true;
             };
 
-            if (!it.done()) ok = load_q();
+            {   // the MMAs only accumulate into S: start from zero
+                uint32_t z[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) z[j] = 0u;
+                for (int i = 0; i < S_SETS; ++i) tmem_st32(tmem + lane_base + S_COL + i * PG + half * 32, z);
+                tmem_wait_st();
+            }
+            if (!it.done()) ok = load_q();  // its barrier also orders the zeroing before q_ready
+            PROF_DECL
             while (ok && !it.done()) {
-                if (t == 0) bulk_wait_read_le1();  // staging slot sg was read by its copy
-                bool w = !pfail && wait(bar(ctrl->s_full[sb.i]), sb.ph, abort_flag);
-                if (!(ok = named_red_and(w, BAR_OK, 128))) break;
+                if (t == 0) TRACE(27, u);
+                if (t == 32) TRACE(67, u);
+                bool good = wait(bar(ctrl->s_full[sb.i]), sb.ph, abort_flag);
+                PROF_MARK(0);
                 if (t == 0) TRACE(5, u);
-                tc_fence_after();
-                float x[64];
+                if (t == 32) TRACE(45, u);
+                float mine[32], other[32];
                 {
-                    uint32_t a0[32], a1[32], b0[32], b1[32];
-                    const uint32_t sa = tmem + lane_base + S_COL + sb.i * 2 * PG;
-                    tmem_ld32(sa, a0);
-                    tmem_ld32(sa + 32, a1);
-                    tmem_ld32(sa + PG, b0);
-                    tmem_ld32(sa + PG + 32, b1);
+                    uint32_t a[32], b[32];
+                    const uint32_t sa = tmem + lane_base + S_COL + sb.i * PG;
+                    tc_fence_after();
+                    tmem_ld32(sa + half * 32, a);
+                    tmem_ld32(sa + (half ^ 1) * 32, b);
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        x[j] = __uint_as_float(a0[j]) + __uint_as_float(b0[j]);
-                        x[32 + j] = __uint_as_float(a1[j]) + __uint_as_float(b1[j]);
+                        mine[j] = __uint_as_float(a[j]);
+                        other[j] = __uint_as_float(b[j]);
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(ctrl->s_free[sb.i]));
+                if (t == 0) TRACE(26, u);
+                if (t == 32) TRACE(66, u);
+                const uint32_t s_buf = sb.i;  // zeroed and released after the vote (all warps have read it)
+                PROF_MARK(1);
                 if (t == 0) TRACE(24, u);
+                if (t == 32) TRACE(64, u);
                 sb.adv(S_SETS);
                 st.adv(KV_STAGES);  // this page's stage
 
                 const bool first = it.first, last = it.last();
                 const int valid = it.valid();
                 const int r = it.r;
-                // The last page's S is complete, so every QK of this segment has finished and
-                // the next segment's Q may overwrite TMEM now.
-                if (last && it.left > 1) {
-                    if (!(ok = load_q())) break;
-                }
-
                 // ---- online softmax (log2 units; scale folded into one FFMA) ----
-                float mraw = -INFINITY;
                 if (valid < PG) {
 #pragma unroll
-                    for (int j = 0; j < 64; ++j)
-                        if (j >= valid) x[j] = -INFINITY;
+                    for (int j = 0; j < 32; ++j) {
+                        if (half * 32 + j >= valid) mine[j] = -INFINITY;
+                        if ((half ^ 1) * 32 + j >= valid) other[j] = -INFINITY;
+                    }
                 }
-#pragma unroll
-                for (int j = 0; j < 64; ++j) mraw = fmaxf(mraw, x[j]);
-                const float mx = mraw * P.scale_log2;
+                const float mx = fmaxf(max32(mine), max32(other)) * P.scale_log2;
                 float m_new = m_used, fac = 1.f;
-                bool need = false;
                 if (first) {
                     m_new = mx;
                     l = 0.f;
                 } else if (mx > m_used + RESCALE_LOG2) {
                     m_new = mx;
                     fac = fast_exp2(m_used - m_new);
-                    need = true;
                 }
-                float sum = 0.f;
-                uint32_t pk[32];
+                float s0 = 0.f, s1 = 0.f;
+                uint32_t pk[16];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float p0 = fast_exp2(fmaf(x[2 * j], P.scale_log2, -m_new));
-                    const float p1 = fast_exp2(fmaf(x[2 * j + 1], P.scale_log2, -m_new));
-                    sum += p0 + p1;
+                for (int j = 0; j < 16; ++j) {
+                    const float p0 = fast_exp2(fmaf(mine[2 * j], P.scale_log2, -m_new));
+                    const float p1 = fast_exp2(fmaf(mine[2 * j + 1], P.scale_log2, -m_new));
+                    s0 += p0;
+                    s1 += p1;
                     pk[j] = pack_bf16x2(p0, p1);
                 }
-                l = l * fac + sum;
+                l = l * fac + (s0 + s1);
                 m_used = m_new;
+                PROF_MARK(2);
                 if (t == 0) TRACE(25, u);
+                if (t == 32) TRACE(65, u);
+                if (last && half) ctrl->lx[seg & 1][h] = l;  // read by the other half after the vote
 
-                // ---- stage P, factors and flag locally; one bulk copy to the PV CTA ----
-                const uint32_t sbase = data_s + STAGE_OFF + sg.i * P_SLOT;
-                const uint32_t rowa = sbase + h * 128;
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    st_shared_v4(rowa + ((c ^ (h & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-                st_shared_u32(sbase + P_FACT + h * 4, __float_as_uint(need ? fac : 1.f));
-                fence_proxy_async_smem();
-                const bool any = named_red_or(need, BAR_FLAG, 128);
-                if (t == 0) {
-                    st_shared_u32(sbase + P_FLAG, any ? 1u : 0u);
-                    fence_proxy_async_smem();
-                    TRACE(9, u);
-                    if (!wait<true>(bar(ctrl->pfree[ps.i]), ps.ph ^ 1u, abort_flag)) {
-                        pfail = true;  // joins the next page's barrier vote, so all threads leave
-                    } else {
-                        bulk_copy_to_peer(p_slot_r[ps.i], sbase, MSG_BYTES, p_full_r[ps.i]);
-                        TRACE(8, u);
-                    }
+                // ---- hand P to the senders through TMEM (one buffer: the senders took the last) ----
+                good = good && wait(bar(ctrl->p_taken), (uint32_t)(u & 1) ^ 1u, abort_flag);
+                PROF_MARK(3);
+                if (t == 0) TRACE(28, u);
+                if (named_red_or(!good, BAR_FAIL, SM_THREADS)) {
+                    ok = false;
+                    break;
                 }
-                ps.adv(P_SLOTS);
-                sg.adv(STAGE_SLOTS);
+                PROF_MARK(4);
+                if (t == 0) TRACE(29, u);
+                tc_fence_after();
+                {   // every softmax warp has read this S buffer: zero my half for its next page
+                    uint32_t z[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) z[j] = 0u;
+                    tmem_st32(tmem + lane_base + S_COL + s_buf * PG + half * 32, z);
+                }
+                tmem_st16(tmem + lane_base + P_COL + half * 16, pk);
+                if (!half) ctrl->fac[u & 1][h] = fac;
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(bar(ctrl->s_free[s_buf]));
+                    mbar_arrive(bar(ctrl->p_ready));
+                }
+                PROF_MARK(5);
+                PROF_PAGE();
+                if (t == 0) TRACE(30, u);
                 ++u;
 
                 if (last) {
-                    const size_t slot = (size_t)pair + r;
-                    P.m_part[slot * NH + h] = m_used;
-                    P.l_part[slot * NH + h] = l;
+                    if (!half) {
+                        const size_t sl = (size_t)pair + r;
+                        P.m_part[sl * NH + h] = m_used;
+                        P.l_part[sl * NH + h] = l + ctrl->lx[seg & 1][h];
+                    }
                     m_used = -INFINITY;
                     l = 0.f;
+                    ++seg;
+                    // The last page's S is complete, so every QK MMA of this segment has finished
+                    // and the next segment's Q may overwrite TMEM now.
+                    if (it.left > 1 && !(ok = load_q())) break;
+                    PROF_MARK(6);
                 }
                 it.next(P);
             }
-            if (t == 0) bulk_wait_all();
-            if (!ok || pfail) fail();
+            if (!ok) fail();
+            PROF_FLUSH();
+        } else if (warp >= SD_WARP0 && warp < SD_WARP0 + 4) {  // senders: P in TMEM -> CTA 1 slot
+            const int t = threadIdx.x - SD_WARP0 * 32;          // 0..127
+            const int quarter = warp & 3;
+            const int h = quarter * 32 + lane;
+            const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+            const uint32_t slot_r = mapa(data_s + P_OFF, 1), p_full_r = mapa(bar(ctrl->p_full[0]), 1);
+            PageIt it;
+            it.init(P, pair);
+            Ring ps{0, 0};
+            int u = 0;
+            bool ok = true;
+            uint32_t sent = 0, sent_ph = 0;  // slots with a message out, and its phase
+            PROF_DECL
+            while (ok && !it.done()) {
+                bool good = wait(bar(ctrl->p_ready), (uint32_t)(u & 1), abort_flag);
+                PROF_MARK(0);
+                good = good && wait<true>(bar(ctrl->pfree[ps.i]), ps.ph ^ 1u, abort_flag);
+                PROF_MARK(5);
+                if (named_red_or(!good, BAR_SFAIL, SD_THREADS)) {
+                    ok = false;
+                    break;
+                }
+                PROF_MARK(1);
+                if (t == 0) TRACE(9, u);
+                tc_fence_after();
+                uint32_t pv[32];
+                tmem_ld32(tmem + lane_base + P_COL, pv);
+                tmem_wait_ld();
+                const float fac = ctrl->fac[u & 1][h];
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(ctrl->p_taken));
+                PROF_MARK(2);
+                const uint32_t slot = slot_r + ps.i * P_SLOT, fb = p_full_r + ps.i * 8;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    st_async_v4(slot + h * 128 + ((c ^ (h & 7)) << 4), pv[4 * c], pv[4 * c + 1], pv[4 * c + 2],
+                                pv[4 * c + 3], fb);
+                st_async_b32(slot + P_FACT + h * 4, __float_as_uint(fac), fb);
+                PROF_MARK(3);
+                const bool any = named_red_or(fac != 1.f, BAR_SFLAG, SD_THREADS);
+                if (t == 0) {
+                    st_async_b32(slot + P_FLAG, any ? 1u : 0u, fb);
+                    sent |= 1u << ps.i;
+                    sent_ph = (sent_ph & ~(1u << ps.i)) | (ps.ph << ps.i);
+                    TRACE(8, u);
+                }
+                PROF_MARK(4);
+                PROF_PAGE();
+                ps.adv(P_SLOTS);
+                ++u;
+                it.next(P);
+            }
+            if (!ok) fail();
+            PROF_FLUSH();
+            // drain: CTA 1's arrivals on our slot barriers (its MMA commits, its readers) for the
+            // messages still out have landed before this CTA can leave
+            if (t == 0)
+                for (int i = 0; i < P_SLOTS; ++i)
+                    if (sent & (1u << i)) wait<true>(bar(ctrl->pfree[i]), (sent_ph >> i) & 1u, never, 10000000ull);
         }
     } else {
         // ===================================== PV CTA =====================================
-        if ((warp == 0 || warp == PROD2_WARP) && lane == 0) {  // TMA producers: content columns
-            const int half = warp == 0 ? 0 : 1;                    // column blocks 4*half .. +3
+        if (warp == 0 && lane == 0) {  // TMA producer: content columns as two half pages
             prefetch_tensormap(&tm_kv4);
             PageIt it;
             it.init(P, pair);
             Ring vs{0, 0};
+            int issued[VH_STAGES];
+            uint32_t nph[VH_STAGES] = {};
+            for (int i = 0; i < VH_STAGES; ++i) issued[i] = 0;
             int u = 0;
             bool ok = true;
-            while (!it.done()) {
-                if (!(ok = wait(bar(ctrl->v_empty[vs.i]), vs.ph ^ 1u, abort_flag))) break;
+            PROF_DECL
+            while (ok && !it.done()) {
                 const int blk = block_of(P, it.r, it.pg);
-                mbar_arrive_expect_tx(bar(ctrl->v_full[vs.i]), V_STAGE / 2);
-                tma_load_3d(data_s + V_OFF + vs.i * V_STAGE + half * 4 * CB, &tm_kv4, 0, blk * PG, half * 4,
-                            bar(ctrl->v_full[vs.i]));
-                if (!half) TRACE(11, u);
+                for (int hh = 0; hh < 2; ++hh) {
+                    PROF_MARK(1);
+                    if (!(ok = wait(bar(ctrl->v_empty[vs.i]), vs.ph ^ 1u, abort_flag))) break;
+                    PROF_MARK(0);
+                    mbar_arrive_expect_tx(bar(ctrl->v_full[vs.i]), VH_STAGE);
+                    tma_load_3d(data_s + V_OFF + vs.i * VH_STAGE, &tm_kv4, 0, blk * PG, hh * 4,
+                                bar(ctrl->v_full[vs.i]));
+                    issued[vs.i] = 1;
+                    nph[vs.i] = vs.ph;
+                    vs.adv(VH_STAGES);
+                }
+                if (!ok) break;
+                PROF_PAGE();
+                TRACE(11, u);
                 ++u;
-                vs.adv(V_STAGES);
                 it.next(P);
             }
             if (!ok) fail();
+            PROF_FLUSH();
+            for (int i = 0; i < VH_STAGES; ++i)
+                if (issued[i]) wait(bar(ctrl->v_full[i]), nph[i], never);
         } else if (warp == 1 && lane == 0) {  // MMA issuer: O += P . V
             constexpr uint32_t idesc = idesc_bf16(128, 256, false, true);
             PageIt it;
             it.init(P, pair);
             Ring vs{0, 0}, ps{0, 0};
             uint32_t ncorr = 0, nseg = 0;
+            uint32_t vr_ph = 0;  // phase bit of v_ready[i]: it completes only on ragged pages
             int u = 0;
-            bool ok = true;
-            while (!it.done()) {
-                if (!(ok = wait(bar(ctrl->v_ready[vs.i]), vs.ph, abort_flag))) break;
-                TRACE(12, u);
+            bool ok = true, any = false;
+            PROF_DECL
+            while (ok && !it.done()) {
+                PROF_MARK(4);
                 if (!(ok = wait<true>(bar(ctrl->p_full[ps.i]), ps.ph, abort_flag))) break;
+                PROF_MARK(0);
                 TRACE(13, u);
                 const uint32_t pa = data_s + P_OFF + ps.i * P_SLOT;
                 const uint32_t flag = ld_shared_u32(pa + P_FLAG);
@@ -627,77 +752,107 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv5, const __grid_consta
                     if (!(ok = wait(bar(ctrl->corr_done), ncorr & 1u, abort_flag))) break;
                     ++ncorr;
                 }
-                const bool first = it.first;
+                const bool first = it.first, ragged = it.valid() < PG;
                 if (first && nseg > 0) {
                     if (!(ok = wait(bar(ctrl->o_free), (nseg - 1) & 1u, abort_flag))) break;
                 }
-                tc_fence_after();
-                const uint32_t vb = data_s + V_OFF + vs.i * V_STAGE;
+                PROF_MARK(1);
+                for (int nh = 0; nh < 2; ++nh) {
+                    PROF_MARK(3);
+                    if (ragged) {
+                        ok = wait(bar(ctrl->v_ready[vs.i]), (vr_ph >> vs.i) & 1u, abort_flag);
+                        vr_ph ^= 1u << vs.i;
+                    } else {
+                        ok = wait(bar(ctrl->v_full[vs.i]), vs.ph, abort_flag);
+                    }
+                    if (!ok) break;
+                    PROF_MARK(2);
+                    if (nh == 0) TRACE(12, u);
+                    tc_fence_after();
+                    const uint32_t vb = data_s + V_OFF + vs.i * VH_STAGE;
 #pragma unroll
-                for (int kk = 0; kk < PG / 16; ++kk)
-#pragma unroll
-                    for (int nh = 0; nh < 2; ++nh) {
+                    for (int kk = 0; kk < PG / 16; ++kk) {
                         const uint64_t a = sdesc_sw128(pa + kk * 32, 16, 1024);
-                        const uint64_t b = sdesc_sw128(vb + nh * 4 * CB + kk * 2048, CB, 1024);
+                        const uint64_t b = sdesc_sw128(vb + kk * 2048, CB, 1024);
                         mma_ss(tmem + nh * 256, a, b, idesc, (first && kk == 0) ? 0u : 1u);
                     }
-                mma_commit(bar(ctrl->v_empty[vs.i]));
+                    mma_commit(bar(ctrl->v_empty[vs.i]));
+                    vs.adv(VH_STAGES);
+                }
+                if (!ok) break;
                 mma_commit(bar(ctrl->pv_done[ps.i]));
+                mma_commit_mc(bar(ctrl->pfree[ps.i]), (uint16_t)1u);  // CTA 0's slot barrier
+                PROF_MARK(3);
+                PROF_PAGE();
+                any = true;
                 TRACE(14, u);
                 ++u;
                 if (it.last()) ++nseg;
-                vs.adv(V_STAGES);
                 ps.adv(P_SLOTS);
                 it.next(P);
             }
             if (!ok) fail();
-        } else if (warp >= 2 && warp <= 5) {  // ragged-page zeroing, lazy rescale, P release, epilogue
-            const int sub = warp & 3;
-            const int h = sub * 32 + lane;
-            const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
-            uint32_t pfree_r[P_SLOTS];
-            for (int i = 0; i < P_SLOTS; ++i) pfree_r[i] = mapa(bar(ctrl->pfree[i]), 0);
+            PROF_FLUSH();
+            if (any) {
+                mma_commit(bar(ctrl->mma_idle[0]));
+                wait(bar(ctrl->mma_idle[0]), 0u, never);
+            }
+            // drain: messages CTA 0 may already have sent land before this CTA can leave
+            if (!ok)
+                for (int i = 0; i < P_SLOTS; ++i) {
+                    wait<true>(bar(ctrl->p_full[ps.i]), ps.ph, never, 1000000ull);
+                    ps.adv(P_SLOTS);
+                }
+        } else if (warp >= EP_WARP0 && warp < EP_WARP0 + 4) {  // ragged zeroing, rescale, epilogue
+            const int quarter = warp & 3;
+            const int h = quarter * 32 + lane;
+            const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+            const uint32_t pfree_r = mapa(bar(ctrl->pfree[0]), 0);
             PageIt it;
             it.init(P, pair);
             Ring vs{0, 0}, ps{0, 0}, prev{0, 0};
             int u = 0;
             bool ok = true;
-            while (!it.done()) {
-                // 1. the V stage: zero token rows past the end of a ragged last page
-                if (!(ok = __all_sync(0xffffffffu, wait(bar(ctrl->v_full[vs.i]), vs.ph, abort_flag)))) break;
-                if (h == 0) TRACE(15, u);
+            PROF_DECL
+            while (ok && !it.done()) {
                 const int valid = it.valid();
+                // 1. ragged last page: zero token rows [valid, 64) of both V halves
                 if (valid < PG) {
-                    const int nz = PG - valid;
-                    const uint32_t vb = data_s + V_OFF + vs.i * V_STAGE;
-                    for (int i = h; i < nz * (DC / 64) * 8; i += 128) {
-                        const int c = i & 7, pr = i >> 3;
-                        const int cb = pr / nz, row = valid + pr % nz;
-                        st_shared_v4(vb + cb * CB + row * 128 + c * 16, 0u, 0u, 0u, 0u);
+                    Ring v2 = vs;
+                    for (int hh = 0; hh < 2; ++hh) {
+                        if (!(ok = __all_sync(0xffffffffu, wait(bar(ctrl->v_full[v2.i]), v2.ph, abort_flag)))) break;
+                        const int nz = PG - valid;
+                        const uint32_t vb = data_s + V_OFF + v2.i * VH_STAGE;
+                        for (int i = h; i < nz * 4 * 8; i += 128) {  // 4 tiles x nz rows x 8 chunks
+                            const int c = i & 7, pr = i >> 3;
+                            const int cb = pr / nz, row = valid + pr % nz;
+                            st_shared_v4(vb + cb * CB + row * 128 + c * 16, 0u, 0u, 0u, 0u);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(ctrl->v_ready[v2.i]));
+                        v2.adv(VH_STAGES);
                     }
-                    fence_proxy_async_smem();
+                    if (!ok) break;
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(ctrl->v_ready[vs.i]));
-                // 2. the P message of this page
+                PROF_MARK(0);
+                // 2. the P message: this head's factor and the flag; then free the slot for reading
                 if (!(ok = __all_sync(0xffffffffu, wait<true>(bar(ctrl->p_full[ps.i]), ps.ph, abort_flag)))) break;
-                if (h == 0) TRACE(16, u);
                 const uint32_t pa = data_s + P_OFF + ps.i * P_SLOT;
                 const float fac = __uint_as_float(ld_shared_u32(pa + P_FACT + h * 4));
                 const uint32_t flag = ld_shared_u32(pa + P_FLAG);
-                const bool first = it.first, last = it.last();
-                // 3. release the previous page's P slot once its PV has completed
-                if (!first) {
-                    if (!(ok = __all_sync(0xffffffffu, wait(bar(ctrl->pv_done[prev.i]), prev.ph, abort_flag)))) break;
-                    if (h == 0) mbar_arrive_remote(pfree_r[prev.i]);
-                    if (h == 0) TRACE(17, u);
-                }
-                // 4. lazy rescale of O rows whose running max moved (PV of the previous page done)
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(pfree_r + ps.i * 8);
+                PROF_MARK(1);
+                if (h == 0) TRACE(16, u);
+                const bool last = it.last();
+                // 3. lazy rescale of O rows whose running max moved (the previous page's PV done)
                 if (flag) {
+                    if (!(ok = __all_sync(0xffffffffu, wait(bar(ctrl->pv_done[prev.i]), prev.ph, abort_flag)))) break;
                     tc_fence_after();
                     if (__any_sync(0xffffffffu, fac != 1.f)) {
 #pragma unroll 1
-                        for (int ch = 0; ch < 16; ++ch) {
+                        for (int ch = 0; ch < DC / 32; ++ch) {
                             uint32_t v[32];
                             tmem_ld32(tmem + lane_base + ch * 32, v);
                             tmem_wait_ld();
@@ -711,44 +866,40 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv5, const __grid_consta
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(ctrl->corr_done));
                 }
-                // 5. end of segment: write the partial O (not normalised) of this row and head
+                PROF_MARK(2);
+                // 4. end of segment: this warp writes its 32 heads of the partial O (not normalised)
+                // as bf16 pairs of columns, [slot][d_c / 2][n_h] words, so that each store
+                // instruction of the warp covers one whole 128-byte line (32 heads, one pair).
                 if (last) {
                     if (!(ok = __all_sync(0xffffffffu, wait(bar(ctrl->pv_done[ps.i]), ps.ph, abort_flag)))) break;
-                    if (h == 0) mbar_arrive_remote(pfree_r[ps.i]);
                     if (h == 0) TRACE(18, u);
                     tc_fence_after();
-                    // O rows -> swizzled staging (one 32-column chunk at a time) -> TMA store, so the
-                    // global writes are whole 128-byte lines instead of one row per thread.
-                    const int orow = (pair + it.r) * NH;
+                    uint32_t *dst = P.o_part + (size_t)(pair + it.r) * (DC / 2) * NH + h;
 #pragma unroll 1
                     for (int ch = 0; ch < DC / 32; ++ch) {
-                        const uint32_t eb = data_s + EPI_OFF + (ch & 1) * EPI_CHUNK;
-                        if (h == 0) bulk_wait_group_read_le1();  // this buffer's previous store has read it
-                        named_sync(BAR_EPI, 128);
                         uint32_t v[32];
                         tmem_ld32(tmem + lane_base + ch * 32, v);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            st_shared_v4(eb + h * 128 + ((c ^ (h & 7)) << 4), v[4 * c], v[4 * c + 1], v[4 * c + 2],
-                                         v[4 * c + 3]);
-                        fence_proxy_async_smem();
-                        named_sync(BAR_EPI, 128);
-                        if (h == 0) tma_store_2d(&tm_o, eb, ch * 32, orow);
+                        for (int j = 0; j < 16; ++j)
+                            __stcg(dst + (size_t)(ch * 16 + j) * NH,
+                                   pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1])));
                     }
-                    if (h == 0) bulk_wait_group_all();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(ctrl->o_free));
                     if (h == 0) TRACE(19, u);
                 }
+                PROF_MARK(3);
+                PROF_PAGE();
                 ++u;
                 prev = ps;
-                vs.adv(V_STAGES);
+                vs.adv(VH_STAGES, 2);
                 ps.adv(P_SLOTS);
                 it.next(P);
             }
             if (!ok && lane == 0) fail();
+            PROF_FLUSH();
         }
     }
 
@@ -775,6 +926,7 @@ schedule_kernel(int s_q, int rows, const int32_t *__restrict__ seq_lens, int max
                 float *m_part, unsigned *err) {
     __shared__ int warp_tot[32];
     __shared__ int carry_s;
+    pdl_trigger();  // the main kernel may start its prologue now
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     if (tid == 0) carry_s = 0;
     __syncthreads();
@@ -855,6 +1007,57 @@ schedule_kernel(int s_q, int rows, const int32_t *__restrict__ seq_lens, int max
     }
 }
 
+// ---- combine: exact log-sum-exp merge of a row's segment partials --------------------------
+// Block (row r, 16-column chunk); thread = head.  For head h with segments s of the row,
+//     M = max_s m_s,  w_s = 2^(m_s - M),  L = sum_s w_s l_s,
+//     o_lat[r,h,c] = sum_s w_s O_s[c,h] / L,   lse[r,h] = (M + log2 L) ln 2.
+// Partials are bf16 pairs of columns, [slot][d_c / 2][n_h] words, so every load instruction of a
+// warp reads one 128-byte line.  Empty slots (m = -inf: a cluster that got none of the row's
+// pages) have weight 0 and are not read.
+constexpr int CMB_COLS = 16;
+__global__ void __launch_bounds__(NH)
+combine_tc_kernel(const int32_t *__restrict__ seg_range, const uint32_t *__restrict__ o_part,
+                  const float *__restrict__ m_part, const float *__restrict__ l_part,
+                  float *__restrict__ o_lat, float *__restrict__ lse, int vec_out) {
+    const int r = blockIdx.x, cc = blockIdx.y, h = threadIdx.x;
+    pdl_wait();  // the partials of the main kernel
+    const int s0 = seg_range[2 * r], s1 = seg_range[2 * r + 1];
+    float M = -INFINITY;
+#pragma unroll 4
+    for (int s = s0; s < s1; ++s) M = fmaxf(M, __ldcg(m_part + (size_t)s * NH + h));
+    float L = 0.f, acc[CMB_COLS];
+#pragma unroll
+    for (int j = 0; j < CMB_COLS; ++j) acc[j] = 0.f;
+#pragma unroll 2
+    for (int s = s0; s < s1; ++s) {
+        const float ms = __ldcg(m_part + (size_t)s * NH + h);
+        const float w = ms == -INFINITY ? 0.f : exp2f(ms - M);
+        if (w == 0.f) continue;  // empty slot (uniform across the block)
+        L = fmaf(w, __ldcg(l_part + (size_t)s * NH + h), L);
+        const uint32_t *src = o_part + ((size_t)s * (DC / 2) + cc * (CMB_COLS / 2)) * NH + h;
+        uint32_t v[CMB_COLS / 2];
+#pragma unroll
+        for (int k = 0; k < CMB_COLS / 2; ++k) v[k] = __ldcg(src + (size_t)k * NH);
+#pragma unroll
+        for (int k = 0; k < CMB_COLS / 2; ++k) {
+            acc[2 * k] = fmaf(w, __uint_as_float(v[k] << 16), acc[2 * k]);
+            acc[2 * k + 1] = fmaf(w, __uint_as_float(v[k] & 0xffff0000u), acc[2 * k + 1]);
+        }
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    float *out = o_lat + ((size_t)r * NH + h) * DC + cc * CMB_COLS;
+    if (vec_out) {  // o_lat 16-byte aligned
+        float4 *dst = reinterpret_cast<float4 *>(out);
+#pragma unroll
+        for (int j = 0; j < CMB_COLS / 4; ++j)
+            dst[j] = make_float4(acc[4 * j] * inv, acc[4 * j + 1] * inv, acc[4 * j + 2] * inv, acc[4 * j + 3] * inv);
+    } else {
+#pragma unroll
+        for (int j = 0; j < CMB_COLS; ++j) out[j] = acc[j] * inv;
+    }
+    if (lse && cc == 0) lse[(size_t)r * NH + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+}
+
 // ---- host side ------------------------------------------------------------------------------
 int g_pairs[64] = {};
 
@@ -888,7 +1091,8 @@ int tc_pairs() {
 }
 
 struct TcWs {
-    float *o, *m, *l;
+    uint32_t *o;  // bf16 pairs
+    float *m, *l;
     int32_t *work, *seg_range, *prefix;
 };
 
@@ -900,14 +1104,14 @@ size_t tc_layout(int pairs, int rows, char *base, TcWs *w) {
         off += align_up(bytes, 256);
         return p;
     };
-    char *o = take(slots * NH * DC * sizeof(float));
+    char *o = take(slots * NH * (DC / 2) * sizeof(uint32_t));
     char *m = take(slots * NH * sizeof(float));
     char *l = take(slots * NH * sizeof(float));
     char *wk = take((size_t)pairs * 4 * sizeof(int32_t));
     char *sr = take((size_t)rows * 2 * sizeof(int32_t));
     char *pf = take(((size_t)rows + 1) * sizeof(int32_t));
     if (w) {
-        w->o = reinterpret_cast<float *>(o);
+        w->o = reinterpret_cast<uint32_t *>(o);
         w->m = reinterpret_cast<float *>(m);
         w->l = reinterpret_cast<float *>(l);
         w->work = reinterpret_cast<int32_t *>(wk);
@@ -931,6 +1135,17 @@ extern "C" int mla_trace_dump(uint32_t *host, int max_entries) {
 }
 #endif
 
+#ifdef MLA_PROF
+// Copies the phase accumulators (2 x 16 x 8 u64) and clears them.
+extern "C" int mla_prof_dump(unsigned long long *host) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+    cudaMemcpyFromSymbol(host, g_prof, sizeof(g_prof));
+    static unsigned long long zeros[2 * 16 * 8];
+    cudaMemcpyToSymbol(g_prof, zeros, sizeof(zeros));
+    return 0;
+}
+#endif
+
 bool tc_supported(const mla_dims_t &d) {
     return d.n_h == NH && d.d_c == DC && d.d_r == ROW - DC && d.page_size == PG &&
            d.act_dtype == MLA_DTYPE_BF16 && d.kv_dtype == MLA_DTYPE_BF16;
@@ -951,13 +1166,11 @@ cudaError_t launch_decode_tc(const mla_dims_t &d, int B, int s_q, const void *q_
     if (pairs < 1) return cudaErrorNotSupported;
     TcWs w;
     if (tc_layout(pairs, rows, reinterpret_cast<char *>(ws), &w) > ws_bytes) return cudaErrorInvalidValue;
-    CUtensorMap tm_kv5, tm_kv4, tm_q4, tm_qr, tm_o;
+    CUtensorMap tm_kv9, tm_kv4, tm_q9;
     const uint64_t pool_rows = (uint64_t)num_blocks * PG, q_rows = (uint64_t)rows * NH;
-    if (!tmap_bf16_colblocks(&tm_kv5, kv_pool, pool_rows, ROW, ROW * 2, PG, SPLIT_LOAD) ||
+    if (!tmap_bf16_colblocks(&tm_kv9, kv_pool, pool_rows, ROW, ROW * 2, PG, NCB) ||
         !tmap_bf16_colblocks(&tm_kv4, kv_pool, pool_rows, ROW, ROW * 2, PG, 4) ||
-        !tmap_bf16_colblocks(&tm_q4, q_abs, q_rows, ROW, ROW * 2, 64, 4) ||
-        !tmap_bf16_2d(&tm_qr, q_abs, ROW, q_rows, ROW * 2, 64, NH) ||
-        !tmap_2d(&tm_o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w.o, DC, ((uint64_t)pairs + rows) * NH, DC * 4, 32, NH))
+        !tmap_bf16_colblocks(&tm_q9, q_abs, q_rows, ROW, ROW * 2, 64, NCB))
         return cudaErrorInvalidValue;
     unsigned *err = device_error_word();
     schedule_kernel<<<1, 1024, 0, st>>>(s_q, rows, seq_lens, max_seq_len, max_blocks, pairs, w.prefix,
@@ -978,11 +1191,30 @@ cudaError_t launch_decode_tc(const mla_dims_t &d, int B, int s_q, const void *q_
     P.l_part = w.l;
     P.scale_log2 = (float)(1.4426950408889634 / sqrt((double)(d.d_h + d.d_r)));
     P.err = err;
-    decode_tc_kernel<<<2 * pairs, THREADS, SMEM_BYTES, st>>>(tm_kv5, tm_kv4, tm_q4, tm_qr, tm_o, P);
-    e = cudaGetLastError();
+    // The main and combine kernels are launched as programmatic dependents of the kernel before
+    // them: their blocks may start while it drains, and they wait for its results on the device.
+    cudaLaunchAttribute pdl;
+    pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl.val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = st;
+    cfg.attrs = &pdl;
+#ifdef MLA_NO_PDL
+    cfg.numAttrs = 0;
+#else
+    cfg.numAttrs = 1;
+#endif
+    e = cudaLaunchKernelEx(&cfg, decode_tc_kernel, tm_kv9, tm_kv4, tm_q9, P);
     if (e != cudaSuccess) return e;
-    Partials part{w.o, w.m, w.l};
-    return launch_combine(rows, NH, DC, part, w.seg_range, 0, o_lat, lse, st);
+    const int vec_out = (reinterpret_cast<uintptr_t>(o_lat) & 15) == 0;
+    cfg.gridDim = dim3(rows, DC / CMB_COLS);
+    cfg.blockDim = dim3(NH);
+    cfg.dynamicSmemBytes = 0;
+    return cudaLaunchKernelEx(&cfg, combine_tc_kernel, (const int32_t *)w.seg_range, (const uint32_t *)w.o,
+                              (const float *)w.m, (const float *)w.l, o_lat, lse, vec_out);
 }
 
 }  // namespace mla

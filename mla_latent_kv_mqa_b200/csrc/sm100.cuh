@@ -75,10 +75,11 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 
 // Bounded wait: gives up after `limit_ns` of wall-clock time or as soon as *abort is set.
 // Returns false on give-up (the caller then leaves its loop; see the kernel's teardown).
-template <bool kCluster = false>
-__device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort,
-                                     uint64_t limit_ns = 2000000000ull) {
-    if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+// The first probe is inline; the polling loop is one out-of-line copy per barrier scope, which
+// keeps the many call sites of a large warp-specialised kernel small in the instruction cache.
+template <bool kCluster>
+__device__ __noinline__ bool wait_poll(uint32_t bar, uint32_t parity, volatile uint32_t *abort,
+                                       uint64_t limit_ns) {
     const uint64_t t0 = globaltimer();
     while (true) {
         if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
@@ -86,6 +87,29 @@ __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, volatile uin
         if (globaltimer() - t0 > limit_ns) return false;
     }
 }
+template <bool kCluster = false>
+__device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort,
+                                     uint64_t limit_ns = 2000000000ull) {
+    if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+#ifdef MLA_WAIT_INLINE
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (globaltimer() - t0 > limit_ns) return false;
+    }
+#else
+    return wait_poll<kCluster>(bar, parity, abort, limit_ns);
+#endif
+}
+
+// ---- programmatic dependent launch ----------------------------------------------------------
+// Wait until the grids this one depends on have completed and their writes are visible (a no-op
+// when the launch had no programmatic dependency).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel in the stream start launching its blocks (its pdl_wait still waits for
+// this grid to complete).
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---- cluster / distributed shared memory -------------------------------------------------
 __device__ __forceinline__ uint32_t mapa(uint32_t local_addr, uint32_t rank) {
@@ -194,6 +218,14 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
         : "memory");
 }
+// Same, but the arrive goes to the mbarrier at this barrier's shared-memory offset in every CTA
+// of the cluster whose bit is set in cta_mask (this CTA included only if its bit is set).
+__device__ __forceinline__ void mma_commit_mc(uint32_t bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::
+            "r"(bar), "h"(cta_mask)
+        : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -222,6 +254,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
         "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
         "%30, %31, %32};" ::"r"(taddr),
         MLA_W8(0), MLA_W8(8), MLA_W8(16), MLA_W8(24)
+        : "memory");
+}
+// 16 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+        "%12, %13, %14, %15, %16};" ::"r"(taddr),
+        MLA_W8(0), MLA_W8(8)
         : "memory");
 }
 #undef MLA_R8
