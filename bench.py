@@ -81,14 +81,15 @@ class ClockSampler:
 
     def __init__(self, bus: int | None):
         self.bus = bus
-        self.rows = []
+        self.rows = []      # (arrival time, fields)
         self.error = None
         self._p = None
+        self.window = None  # (t0, t1): summarise only samples that arrived in it
 
     def __enter__(self):
         try:
             self._p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                                        "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
+                                        "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
             self._t = threading.Thread(target=self._read, daemon=True)
             self._t.start()
         except OSError as e:
@@ -106,7 +107,7 @@ class ClockSampler:
             except (IndexError, ValueError):
                 bus = None
             if self.bus is None or bus == self.bus:
-                self.rows.append(r)
+                self.rows.append((time.time(), r))
 
     def __exit__(self, *a):
         if self._p:
@@ -119,16 +120,20 @@ class ClockSampler:
                 self._p.kill()
 
     def summary(self):
-        if not self.rows:
+        rows = [r for t, r in self.rows
+                if self.window is None or self.window[0] <= t <= self.window[1]]
+        if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0,
                     "error": self.error}
+        self.rows = [(0.0, r) for r in rows]
         num = lambda x: float(x) if x.replace(".", "", 1).isdigit() else None
-        sm = [v for v in (num(r[1]) for r in self.rows) if v is not None]
-        mx = [v for v in (num(r[2]) for r in self.rows) if v is not None]
-        pw = [v for v in (num(r[3]) for r in self.rows) if v is not None]
-        reasons = sorted({self.NAMES[i] for r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
+        sm = [v for v in (num(r[1]) for _, r in self.rows) if v is not None]
+        mx = [v for v in (num(r[2]) for _, r in self.rows) if v is not None]
+        pw = [v for v in (num(r[3]) for _, r in self.rows) if v is not None]
+        reasons = sorted({self.NAMES[i] for _, r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "power_w_max": max(pw) if pw else None, "reasons": reasons, "samples": len(self.rows)}
+                "power_w_max": max(pw) if pw else None, "reasons": reasons, "samples": len(self.rows),
+                "window": "the last 0.5 s of the sustained warm-up load and the timed region"}
 
 
 def cpu_baseline(wl, budget_s: float = 12.0):
@@ -272,21 +277,22 @@ def run_mine(args):
             g_dec.replay()
             g_e2e.replay()
         stream.synchronize()
-        # let the SM clock ramp up under sustained load before timing (idle boards sit far below boost)
-        t_end = time.time() + args.clock_warmup_s
-        while time.time() < t_end:
-            for _ in range(20):
-                g_step.replay()
-            stream.synchronize()
-
         K = args.steps
         mk = lambda: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
         ev, dev_ev, e2e_ev = mk(), mk(), mk()
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
         bus = torch.cuda.get_device_properties(dev).pci_bus_id
         with ClockSampler(bus) as clk:
+            # let the SM clock ramp up under sustained load before timing (idle boards sit far below
+            # boost); the clock samples of its last half second count with the timed region's
+            t_end = time.time() + max(args.clock_warmup_s, 0.8)
+            while time.time() < t_end:
+                for _ in range(20):
+                    g_step.replay()
+                stream.synchronize()
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            t_timed = time.time()
             for k in range(K):
                 flush.fill_(k & 0xFF)
                 ev[k][0].record(stream)
@@ -307,6 +313,8 @@ def run_mine(args):
                 e2e_ev[k][1].record(stream)
                 stream.synchronize()
                 _ = float(h_out[0, 0, 0])  # the host reads the step's result
+            clk.window = (t_timed - 0.5, time.time() + 0.15)
+            time.sleep(0.15)  # the sample in flight at the end
     step_ms = sum(a.elapsed_time(b) for a, b in ev) / K
     dec_ms = sum(a.elapsed_time(b) for a, b in dev_ev) / K
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / K

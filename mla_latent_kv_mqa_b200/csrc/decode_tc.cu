@@ -138,14 +138,16 @@ __device__ __forceinline__ int row_tokens(const Params &P, int r) {
 }
 
 // Walks one cluster's pages in order; every role of both CTAs walks the same sequence.
+// The next row's length is loaded one row ahead, so a segment change does not wait on memory.
 struct PageIt {
-    int r, pg, left, nv, np;
+    int r, pg, left, nv, np, nv_next;
     bool first;
     __device__ void init(const Params &P, int pair) {
         r = P.work[4 * pair];
         pg = P.work[4 * pair + 1];
         left = P.work[4 * pair + 2];
         nv = row_tokens(P, r);
+        nv_next = row_tokens(P, r + 1);
         np = (nv + PG - 1) / PG;
         if (np == 0 || pg >= np) left = 0;
         first = true;
@@ -161,7 +163,8 @@ struct PageIt {
             pg = 0;
             do {
                 ++r;
-                nv = row_tokens(P, r);
+                nv = nv_next;
+                nv_next = row_tokens(P, r + 1);
                 np = (nv + PG - 1) / PG;
             } while (left > 0 && np == 0 && r < P.rows);
             if (r >= P.rows) left = 0;
@@ -920,13 +923,16 @@ __device__ __forceinline__ long long unit_start(int c, long long U, int pairs) {
     return (long long)c * U / pairs;
 }
 
+constexpr int kSchedSmemRows = 4096;
 __global__ void __launch_bounds__(1024)
 schedule_kernel(int s_q, int rows, const int32_t *__restrict__ seq_lens, int max_seq_len,
                 int max_blocks, int pairs, int32_t *prefix, int32_t *work, int32_t *seg_range,
                 float *m_part, unsigned *err) {
     __shared__ int warp_tot[32];
     __shared__ int carry_s;
+    __shared__ int pre_s[kSchedSmemRows + 1];  // the prefix, when it fits (searched below)
     pdl_trigger();  // the main kernel may start its prologue now
+    const bool in_smem = rows <= kSchedSmemRows;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     if (tid == 0) carry_s = 0;
     __syncthreads();
@@ -962,16 +968,23 @@ schedule_kernel(int s_q, int rows, const int32_t *__restrict__ seq_lens, int max
         __syncthreads();
         const int incl = x + (wid > 0 ? warp_tot[wid - 1] : 0);
         const int carry = carry_s;
-        if (r < rows) prefix[r] = carry + incl - n;
+        if (r < rows) {
+            prefix[r] = carry + incl - n;
+            if (in_smem) pre_s[r] = carry + incl - n;
+        }
         __syncthreads();
         if (tid == 1023) carry_s = carry + incl;
         __syncthreads();
     }
-    if (tid == 0) prefix[rows] = carry_s;
+    if (tid == 0) {
+        prefix[rows] = carry_s;
+        if (in_smem) pre_s[rows] = carry_s;
+    }
     // Every partial slot starts empty: a row's slot range also spans clusters that got none of
     // its pages (when there are fewer pages than clusters), and the combine must skip those.
     for (size_t i = tid; i < ((size_t)pairs + rows) * NH; i += 1024) m_part[i] = -INFINITY;
     __syncthreads();
+    const int *pre = in_smem ? pre_s : prefix;
     const long long U = carry_s;
     for (int c = tid; c < pairs; c += 1024) {
         const long long s0 = unit_start(c, U, pairs), s1 = unit_start(c + 1, U, pairs);
@@ -980,17 +993,17 @@ schedule_kernel(int s_q, int rows, const int32_t *__restrict__ seq_lens, int max
             int lo = 0, hi = rows - 1;
             while (lo < hi) {
                 const int mid = (lo + hi + 1) >> 1;
-                if (prefix[mid] <= s0) lo = mid; else hi = mid - 1;
+                if (pre[mid] <= s0) lo = mid; else hi = mid - 1;
             }
             r0 = lo;
         }
         work[4 * c + 0] = r0;
-        work[4 * c + 1] = s1 > s0 ? (int)(s0 - prefix[r0]) : 0;
+        work[4 * c + 1] = s1 > s0 ? (int)(s0 - pre[r0]) : 0;
         work[4 * c + 2] = (int)(s1 - s0);
         work[4 * c + 3] = 0;
     }
     for (int r = tid; r < rows; r += 1024) {
-        const long long u0 = prefix[r], u1 = prefix[r + 1];
+        const long long u0 = pre[r], u1 = pre[r + 1];
         if (u1 <= u0) {
             seg_range[2 * r] = 0;
             seg_range[2 * r + 1] = 0;
@@ -1015,6 +1028,7 @@ schedule_kernel(int s_q, int rows, const int32_t *__restrict__ seq_lens, int max
 // warp reads one 128-byte line.  Empty slots (m = -inf: a cluster that got none of the row's
 // pages) have weight 0 and are not read.
 constexpr int CMB_COLS = 16;
+constexpr int CMB_FAST = 8;  // rows split over at most this many slots take the fast path
 __global__ void __launch_bounds__(NH)
 combine_tc_kernel(const int32_t *__restrict__ seg_range, const uint32_t *__restrict__ o_part,
                   const float *__restrict__ m_part, const float *__restrict__ l_part,
@@ -1022,26 +1036,58 @@ combine_tc_kernel(const int32_t *__restrict__ seg_range, const uint32_t *__restr
     const int r = blockIdx.x, cc = blockIdx.y, h = threadIdx.x;
     pdl_wait();  // the partials of the main kernel
     const int s0 = seg_range[2 * r], s1 = seg_range[2 * r + 1];
-    float M = -INFINITY;
-#pragma unroll 4
-    for (int s = s0; s < s1; ++s) M = fmaxf(M, __ldcg(m_part + (size_t)s * NH + h));
-    float L = 0.f, acc[CMB_COLS];
+    float M = -INFINITY, L = 0.f, acc[CMB_COLS];
 #pragma unroll
     for (int j = 0; j < CMB_COLS; ++j) acc[j] = 0.f;
+    if (s1 - s0 <= CMB_FAST) {
+        // Common case: all loads of the row's slots are issued before any is used.
+        float ms[CMB_FAST], ls[CMB_FAST];
+        uint32_t v[CMB_FAST][CMB_COLS / 2];
+#pragma unroll
+        for (int i = 0; i < CMB_FAST; ++i) {
+            const int s = s0 + i;
+            ms[i] = -INFINITY;
+            ls[i] = 0.f;
+            if (s < s1) {
+                ms[i] = __ldcg(m_part + (size_t)s * NH + h);
+                ls[i] = __ldcg(l_part + (size_t)s * NH + h);
+                const uint32_t *src = o_part + ((size_t)s * (DC / 2) + cc * (CMB_COLS / 2)) * NH + h;
+#pragma unroll
+                for (int k = 0; k < CMB_COLS / 2; ++k) v[i][k] = __ldcg(src + (size_t)k * NH);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < CMB_FAST; ++i) M = fmaxf(M, ms[i]);
+#pragma unroll
+        for (int i = 0; i < CMB_FAST; ++i) {
+            // empty slots (m = -inf) and slots past the row's range have weight 0: their (never
+            // written) partials must not enter the sums, not even as 0 * NaN
+            if (ms[i] == -INFINITY) continue;
+            const float w = exp2f(ms[i] - M);
+            L = fmaf(w, ls[i], L);
+#pragma unroll
+            for (int k = 0; k < CMB_COLS / 2; ++k) {
+                acc[2 * k] = fmaf(w, __uint_as_float(v[i][k] << 16), acc[2 * k]);
+                acc[2 * k + 1] = fmaf(w, __uint_as_float(v[i][k] & 0xffff0000u), acc[2 * k + 1]);
+            }
+        }
+    } else {
+        for (int s = s0; s < s1; ++s) M = fmaxf(M, __ldcg(m_part + (size_t)s * NH + h));
 #pragma unroll 2
-    for (int s = s0; s < s1; ++s) {
-        const float ms = __ldcg(m_part + (size_t)s * NH + h);
-        const float w = ms == -INFINITY ? 0.f : exp2f(ms - M);
-        if (w == 0.f) continue;  // empty slot (uniform across the block)
-        L = fmaf(w, __ldcg(l_part + (size_t)s * NH + h), L);
-        const uint32_t *src = o_part + ((size_t)s * (DC / 2) + cc * (CMB_COLS / 2)) * NH + h;
-        uint32_t v[CMB_COLS / 2];
+        for (int s = s0; s < s1; ++s) {
+            const float ms = __ldcg(m_part + (size_t)s * NH + h);
+            if (ms == -INFINITY) continue;  // empty slot (uniform across the block)
+            const float w = exp2f(ms - M);
+            L = fmaf(w, __ldcg(l_part + (size_t)s * NH + h), L);
+            const uint32_t *src = o_part + ((size_t)s * (DC / 2) + cc * (CMB_COLS / 2)) * NH + h;
+            uint32_t v[CMB_COLS / 2];
 #pragma unroll
-        for (int k = 0; k < CMB_COLS / 2; ++k) v[k] = __ldcg(src + (size_t)k * NH);
+            for (int k = 0; k < CMB_COLS / 2; ++k) v[k] = __ldcg(src + (size_t)k * NH);
 #pragma unroll
-        for (int k = 0; k < CMB_COLS / 2; ++k) {
-            acc[2 * k] = fmaf(w, __uint_as_float(v[k] << 16), acc[2 * k]);
-            acc[2 * k + 1] = fmaf(w, __uint_as_float(v[k] & 0xffff0000u), acc[2 * k + 1]);
+            for (int k = 0; k < CMB_COLS / 2; ++k) {
+                acc[2 * k] = fmaf(w, __uint_as_float(v[k] << 16), acc[2 * k]);
+                acc[2 * k + 1] = fmaf(w, __uint_as_float(v[k] & 0xffff0000u), acc[2 * k + 1]);
+            }
         }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
