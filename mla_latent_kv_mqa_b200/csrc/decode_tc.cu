@@ -986,6 +986,85 @@ schedule_kernel(int s_q, int rows, const int32_t *__restrict__ seq_lens, int max
     __syncthreads();
     const int *pre = in_smem ? pre_s : prefix;
     const long long U = carry_s;
+    // ---- row-aligned split: every cluster works on one row only, rows get clusters in
+    // proportion to their pages.  A cluster that crosses a row boundary pays a Q reload, a
+    // drain of its pipeline and a second partial write; this split avoids that whenever it is
+    // as balanced as the contiguous one (e.g. every row fits in whole clusters' shares).
+    if (rows <= pairs && rows <= 1024 && in_smem && U > 0) {
+        __shared__ int k_s[1024], cf_s[1025];
+        __shared__ int red_s[32];
+        __shared__ int ok_s, kbase_s, maxload_s;
+        const int r = tid;
+        const int n = r < rows ? pre_s[r + 1] - pre_s[r] : 0;
+        int k = n > 0 ? (int)max(1LL, (long long)n * pairs / U) : 0;
+        // sum of the base counts
+        int x = k;
+        for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        if (lane == 0) red_s[wid] = x;
+        if (tid == 0) { ok_s = 1; maxload_s = 0; }
+        __syncthreads();
+        if (tid == 0) {
+            int s = 0;
+            for (int i = 0; i < 32; ++i) s += red_s[i];
+            kbase_s = s;
+        }
+        if (r < rows) k_s[r] = k;
+        __syncthreads();
+        const int extra = pairs - kbase_s;
+        if (extra >= 0) {
+            // one more cluster for the `extra` rows with the highest load per cluster (ties: lower row)
+            if (r < rows && n > 0 && extra > 0) {
+                const long long my = (long long)n * 1000000 / k;
+                int rank = 0;
+                for (int i = 0; i < rows; ++i) {
+                    const int ni = pre_s[i + 1] - pre_s[i];
+                    if (ni == 0 || i == r) continue;
+                    const long long li = (long long)ni * 1000000 / k_s[i];
+                    if (li > my || (li == my && i < r)) ++rank;
+                }
+                if (rank < extra) k += 1;
+            }
+            __syncthreads();
+            if (r < rows) {
+                k = min(k, max(n, 0));  // no cluster without pages
+                k_s[r] = k;
+                if (k > 0) atomicMax(&maxload_s, (n + k - 1) / k);
+            }
+            __syncthreads();
+            // accept only if no cluster gets more pages than under the contiguous split: measured
+            // on the uniform batches, a few extra pages cost more than a row change does
+            if (tid == 0) {
+                const long long bal = (U + pairs - 1) / pairs;
+                ok_s = (long long)maxload_s <= bal;
+                int c = 0;
+                for (int i = 0; i < rows; ++i) { cf_s[i] = c; c += k_s[i]; }
+                cf_s[rows] = c;
+            }
+            __syncthreads();
+            if (ok_s) {
+                if (r < rows) {
+                    const int c0 = cf_s[r];
+                    for (int j = 0; j < k; ++j) {
+                        const int p0 = (int)((long long)j * n / k), p1 = (int)((long long)(j + 1) * n / k);
+                        work[4 * (c0 + j) + 0] = r;
+                        work[4 * (c0 + j) + 1] = p0;
+                        work[4 * (c0 + j) + 2] = p1 - p0;
+                        work[4 * (c0 + j) + 3] = 0;
+                    }
+                    seg_range[2 * r] = k > 0 ? c0 + r : 0;
+                    seg_range[2 * r + 1] = k > 0 ? c0 + k + r : 0;
+                }
+                for (int c = cf_s[rows] + tid; c < pairs; c += 1024) {  // idle clusters
+                    work[4 * c + 0] = 0;
+                    work[4 * c + 1] = 0;
+                    work[4 * c + 2] = 0;
+                    work[4 * c + 3] = 0;
+                }
+                return;
+            }
+        }
+    }
+    // ---- contiguous split (any row count)
     for (int c = tid; c < pairs; c += 1024) {
         const long long s0 = unit_start(c, U, pairs), s1 = unit_start(c + 1, U, pairs);
         int r0 = 0;

@@ -18,6 +18,33 @@ def max_abs(x, ref) -> float:
     return float(np.max(np.abs(np.asarray(x, dtype=np.float64) - np.asarray(ref, dtype=np.float64))))
 
 
+# Tolerances (see test_gpu_parity.py's module docstring for their reading).
+BF16_REL, BF16_ABS, FP8_REL, LSE_ABS = 4e-3, 2e-2, 3e-2, 1e-2
+
+
+def scaled_max_abs(x, ref):
+    """max |x - ref| / max(1, max |ref|)."""
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    return float(np.abs(x - ref).max() / max(1.0, float(np.abs(ref).max())))
+
+
+def check_step(got, ref, rows, heads, rel_tol, abs_tol):
+    """Compare one step's (o_lat, lse, o) on the given rows and heads with the oracle's."""
+    q_abs, o_lat, lse, o = got
+    o_lat = o_lat.cpu().numpy()[rows][:, heads]
+    o = o.float().cpu().numpy()[rows][:, heads]
+    lse = lse.cpu().numpy()[rows][:, heads]
+    e = dict(o_lat_rel=rel_l2(o_lat, ref.o_lat), o_rel=rel_l2(o, ref.o),
+             o_lat_abs=scaled_max_abs(o_lat, ref.o_lat), o_abs=scaled_max_abs(o, ref.o),
+             lse_abs=float(np.max(np.abs(lse - ref.lse) / np.maximum(1.0, np.abs(ref.lse)))))
+    assert e["o_lat_rel"] <= rel_tol and e["o_rel"] <= rel_tol, e
+    if abs_tol is not None:
+        assert e["o_lat_abs"] <= abs_tol and e["o_abs"] <= abs_tol, e
+    assert e["lse_abs"] <= LSE_ABS, e
+    return e
+
+
 def _act(x: np.ndarray, act: str, dev):
     t = torch.from_numpy(np.ascontiguousarray(x))
     return t.to(device=dev, dtype=torch.bfloat16 if act == "bf16" else torch.float32)

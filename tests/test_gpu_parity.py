@@ -15,11 +15,11 @@ import pytest
 import torch
 
 from mla_latent_kv_mqa_b200 import workloads as W
-from tests.harness import GpuRun, max_abs, oracle_ref, rel_l2
+from tests.harness import (BF16_ABS, BF16_REL, FP8_REL, LSE_ABS, GpuRun, check_step, max_abs, oracle_ref,
+                           rel_l2, scaled_max_abs)
 
 pytestmark = pytest.mark.gpu
 
-BF16_REL, BF16_ABS, FP8_REL, LSE_ABS = 4e-3, 2e-2, 3e-2, 1e-2
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -31,26 +31,8 @@ def _cuda():
     torch.backends.cuda.matmul.allow_tf32 = False
 
 
-def scaled_max_abs(x, ref):
-    """max |x - ref| / max(1, max |ref|)."""
-    x = np.asarray(x, dtype=np.float64)
-    ref = np.asarray(ref, dtype=np.float64)
-    return float(np.abs(x - ref).max() / max(1.0, float(np.abs(ref).max())))
-
-
 def _check(wl, got, ref, rows, heads, rel_tol, abs_tol):
-    q_abs, o_lat, lse, o = got
-    o_lat = o_lat.cpu().numpy()[rows][:, heads]
-    o = o.float().cpu().numpy()[rows][:, heads]
-    lse = lse.cpu().numpy()[rows][:, heads]
-    e = dict(o_lat_rel=rel_l2(o_lat, ref.o_lat), o_rel=rel_l2(o, ref.o),
-             o_lat_abs=scaled_max_abs(o_lat, ref.o_lat), o_abs=scaled_max_abs(o, ref.o),
-             lse_abs=float(np.max(np.abs(lse - ref.lse) / np.maximum(1.0, np.abs(ref.lse)))))
-    assert e["o_lat_rel"] <= rel_tol and e["o_rel"] <= rel_tol, e
-    if abs_tol is not None:
-        assert e["o_lat_abs"] <= abs_tol and e["o_abs"] <= abs_tol, e
-    assert e["lse_abs"] <= LSE_ABS, e
-    return e
+    return check_step(got, ref, rows, heads, rel_tol, abs_tol)
 
 
 # ---------------------------------------------------------------------------------------------
@@ -63,6 +45,8 @@ SMALL = {
     "v3_lognormal": dict(seed=23, seq_lens=[3000], lognormal_tokens=True),
     "fp8_sq2": dict(seed=24, seq_lens=[300, 2, 65, 128], s_q=2, kv_dtype="fp8"),
     "bf16_sq2": dict(seed=25, seq_lens=[513, 3], s_q=2),
+    # more query rows than the tensor-core kernel has clusters: the scheduler's contiguous split
+    "many_rows": dict(seed=26, seq_lens=[int(x) for x in np.random.default_rng(26).integers(1, 300, 96)]),
 }
 
 
