@@ -401,8 +401,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             // Thread 1 issues a page's part only after thread 0 has issued its own (k0_done, with
             // the tcgen05 thread-sync fences on both sides), so every page sums in the same order
             // and results are bitwise reproducible; thread 0 meanwhile goes on to the next page.
-            constexpr uint32_t idesc = idesc_bf16(128, PG, false, false);
+            // (Splitting by tokens instead -- N = 32 per thread over the whole K, into separate
+            // columns -- needs no ordering but doubles each thread's MMA count; measured slower.)
             const int part = warp - 1;
+            constexpr uint32_t idesc = idesc_bf16(128, PG, false, false);
             const int cb0 = part ? 5 : 0, cb1 = part ? NCB : 5;
             PageIt it;
             it.init(P, pair);
