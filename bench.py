@@ -41,10 +41,10 @@ WORKLOADS = {
 FLUSH_BYTES = 512 << 20
 
 
-def make_workload(name: str):
+def make_workload(name: str, batch: int | None = None):
     from mla_latent_kv_mqa_b200 import workloads as W
     if name == "v3":
-        return W.v3_decode()
+        return W.v3_decode(B=batch or 16)
     if name == "varlen":
         return W.varlen_decode()
     if name == "long":
@@ -370,6 +370,21 @@ def run_mine(args):
         dist.destroy_process_group()
 
 
+def run_plain(args):
+    """--plain-steps N: N eager (non-graph, untimed) steps of the workload, then exit 0.  The
+    command profilers (ncu) are pointed at; --batch overrides the v3 batch, e.g. 32 so that the
+    cache (151 MB) exceeds the 126 MB L2."""
+    import torch
+    from tests.harness import GpuRun
+    wl = make_workload(args.config, args.batch)
+    run = GpuRun(wl)
+    run.fill_cache()
+    for _ in range(args.plain_steps):
+        run.step()
+    torch.cuda.synchronize()
+    print(f"plain steps done: {args.plain_steps} x {wl.name}")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -379,8 +394,12 @@ def main():
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
     ap.add_argument("--config", default="v3", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--plain-steps", type=int, default=0, help="run N untimed eager steps and exit (profiling)")
+    ap.add_argument("--batch", type=int, default=None, help="with --plain-steps: batch of the v3 workload")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.plain_steps:
+        run_plain(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_mine(args)

@@ -31,9 +31,10 @@
 // QK : PV work is 576 : 512, so the two tensor pipes are nearly balanced and no FLOP or byte
 // is done twice (the second read of a page is an L2 hit).
 //
-// Split-KV.  A tiny scheduler kernel spreads all (query row, page) units evenly over the
-// clusters; a cluster's contiguous range may cover parts of several query rows, each part a
-// segment whose (O, m, l) partial is merged exactly by the log-sum-exp combine kernel.
+// Split-KV.  All (query row, page) units are spread evenly over the clusters (each cluster
+// works out its own contiguous range in its prologue, see schedule()); a range may cover parts
+// of several query rows, each part a segment whose (O, m, l) partial is merged exactly by the
+// log-sum-exp combine kernel.
 //
 // Lazy rescaling (log2 units): a row's running max only moves when a page's max exceeds it by
 // more than 8, so P stays <= 256 and O rows are rescaled only on those (rare) pages.
@@ -111,6 +112,8 @@ struct __align__(8) Ctrl {
     uint32_t tmem_base;
     uint32_t abort;
     uint32_t never;             // stays 0: the abort word of drain waits, which must not give up early
+    int w_r0, w_pg0, w_n;       // this cluster's work: first row, first page of it, number of pages
+    int scan[THREADS / 32 + 1]; // scheduling scratch (warp totals)
     float lx[2][NH];            // QK CTA: the second softmax half's row sums, by segment parity
     float fac[2][NH];           // QK CTA: per-head rescale factors of a page, by page parity
 };
@@ -122,7 +125,8 @@ struct Params {
     int max_blocks, num_blocks;
     const int32_t *seq_lens;
     int s_q, rows, max_seq_len;
-    const int32_t *work;  // [pairs][4]: first row, first page, number of pages
+    int pairs;            // clusters of the grid
+    int32_t *seg_range;   // [rows][2]: the row's slot range, written by cluster 0
     uint32_t *o_part;  // [slot][d_c / 2][n_h]: bf16 pairs of columns (c = 2k, 2k + 1) per head
     float *m_part, *l_part;
     float scale_log2;
@@ -142,10 +146,10 @@ __device__ __forceinline__ int row_tokens(const Params &P, int r) {
 struct PageIt {
     int r, pg, left, nv, np, nv_next;
     bool first;
-    __device__ void init(const Params &P, int pair) {
-        r = P.work[4 * pair];
-        pg = P.work[4 * pair + 1];
-        left = P.work[4 * pair + 2];
+    __device__ void init(const Params &P, const int *work) {
+        r = work[0];
+        pg = work[1];
+        left = work[2];
         nv = row_tokens(P, r);
         nv_next = row_tokens(P, r + 1);
         np = (nv + PG - 1) / PG;
@@ -276,12 +280,98 @@ __device__ unsigned long long g_prof[2][16][8];
 #define PROF_FLUSH() ((void)0)
 #endif
 
+// ---- the cluster's share of the work (every CTA computes it; cluster 0 also writes the
+// per-row slot ranges the combine kernel reads) --------------------------------------------
+// All (query row, page) units are numbered row by row; cluster c takes units
+// [c U / pairs, (c + 1) U / pairs).  A row's partial results go to slots c + r of the clusters c
+// that hold its units; a cluster that holds none (possible when there are fewer units than
+// clusters) but sits inside a row's slot range marks its slot empty (m = -inf).
+__device__ __forceinline__ long long unit_start(long long c, long long U, int pairs) { return c * U / pairs; }
+__device__ __forceinline__ int pages_of_row(const Params &P, int r, bool &bad) {
+    const int b = r / P.s_q, i = r - b * P.s_q;
+    const int L = P.seq_lens[b];
+    if (L < P.s_q || L > P.max_seq_len || L > P.max_blocks * PG) {
+        bad |= i == 0;
+        return 0;
+    }
+    return (L - P.s_q + i + 1 + PG - 1) / PG;
+}
+// Block-wide inclusive scan (THREADS threads); returns this thread's inclusive value and sets
+// total.  Uses ctrl->scan; ends with a barrier, so it can be called again right away.
+__device__ __forceinline__ long long block_scan(int x, Ctrl *ctrl, long long &total) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) ctrl->scan[wid] = x;
+    __syncthreads();
+    long long before = 0, all = 0;
+    for (int w = 0; w < THREADS / 32; ++w) {
+        const int v = ctrl->scan[w];
+        if (w < wid) before += v;
+        all += v;
+    }
+    total = all;
+    __syncthreads();
+    return before + x;
+}
+__device__ __noinline__ void schedule(const Params &P, int pair, uint32_t rank, Ctrl *ctrl) {
+    const int tid = threadIdx.x;
+    bool bad = false;
+    long long U = 0;
+    for (int base = 0; base < P.rows; base += THREADS) {  // pass 1: all units
+        const int r = base + tid;
+        long long chunk;
+        block_scan(r < P.rows ? pages_of_row(P, r, bad) : 0, ctrl, chunk);
+        U += chunk;
+    }
+    if (bad && pair == 0 && rank == 0) record_error(P.err, kErrBadSeqLen);
+    const long long s0 = unit_start(pair, U, P.pairs), s1 = unit_start(pair + 1, U, P.pairs);
+    if (tid == 0) {
+        ctrl->w_r0 = 0;
+        ctrl->w_pg0 = 0;
+        ctrl->w_n = (int)(s1 - s0);
+    }
+    __syncthreads();
+    long long carry = 0;
+    for (int base = 0; base < P.rows; base += THREADS) {  // pass 2: locate s0, slot ranges
+        const int r = base + tid;
+        bool b2 = false;
+        const int n = r < P.rows ? pages_of_row(P, r, b2) : 0;
+        long long chunk;
+        const long long u0 = carry + block_scan(n, ctrl, chunk) - n;  // this row's first unit
+        if (n > 0 && u0 <= s0 && s0 < u0 + n) {  // the row holding unit s0
+            if (s1 > s0) {
+                ctrl->w_r0 = r;
+                ctrl->w_pg0 = (int)(s0 - u0);
+            } else if (rank == 0) {
+                // no units here, but this cluster's slot lies inside row r's slot range
+                for (int h = 0; h < NH; ++h) P.m_part[((size_t)pair + r) * NH + h] = -INFINITY;
+            }
+        }
+        if (pair == 0 && rank == 0 && r < P.rows) {
+            auto pair_of = [&](long long u) {  // the cluster holding unit u
+                int c = (int)(u * P.pairs / U);
+                while (c + 1 < P.pairs && unit_start(c + 1, U, P.pairs) <= u) ++c;
+                while (c > 0 && unit_start(c, U, P.pairs) > u) --c;
+                return c;
+            };
+            P.seg_range[2 * r] = n > 0 ? pair_of(u0) + r : 0;
+            P.seg_range[2 * r + 1] = n > 0 ? pair_of(u0 + n - 1) + r + 1 : 0;
+        }
+        carry += chunk;
+    }
+    __syncthreads();
+}
+
 // Named barriers: the 256 softmax threads and the 128 sender threads (QK CTA).
 constexpr int BAR_FAIL = 1, BAR_Q = 2, BAR_SFAIL = 3, BAR_SFLAG = 4;
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_constant__ CUtensorMap tm_kv4,
-                 const __grid_constant__ CUtensorMap tm_q9, const Params P) {
+                 const __grid_constant__ CUtensorMap tm_q9, const __grid_constant__ Params P) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_u32(smem_raw);
     const uint32_t data_s = (raw_s + 1023u) & ~1023u;
@@ -337,9 +427,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
     __syncthreads();
     tc_fence_after();
     cluster_sync();
-    // Everything above overlaps the scheduler kernel; its work list is read from here on.
+    // Everything above overlaps the kernel before this one; inputs are read from here on.
     pdl_trigger();
     pdl_wait();
+    schedule(P, pair, rank, ctrl);
     const uint32_t tmem = ctrl->tmem_base;
     const uint32_t peer = rank ^ 1u;
     if (threadIdx.x == 0) TRACE(20 + rank, (uint32_t)clock64() >> 8);
@@ -359,7 +450,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             prefetch_tensormap(&tm_kv9);
             prefetch_tensormap(&tm_q9);
             PageIt it;
-            it.init(P, pair);
+            it.init(P, &ctrl->w_r0);
             Ring st{0, 0};
             int issued[KV_STAGES];           // phase + 1 of the last copy into each stage (0: none)
             for (int i = 0; i < KV_STAGES; ++i) issued[i] = 0;
@@ -407,7 +498,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             constexpr uint32_t idesc = idesc_bf16(128, PG, false, false);
             const int cb0 = part ? 5 : 0, cb1 = part ? NCB : 5;
             PageIt it;
-            it.init(P, pair);
+            it.init(P, &ctrl->w_r0);
             Ring st{0, 0}, sb{0, 0};
             uint32_t qn = 0;
             int u = 0;
@@ -468,7 +559,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             const int h = quarter * 32 + lane;                  // head = TMEM lane
             const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
             PageIt it;
-            it.init(P, pair);
+            it.init(P, &ctrl->w_r0);
             Ring st{0, 0}, sb{0, 0};
             float m_used = -INFINITY, l = 0.f;
             int u = 0, seg = 0;
@@ -645,7 +736,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
             const uint32_t slot_r = mapa(data_s + P_OFF, 1), p_full_r = mapa(bar(ctrl->p_full[0]), 1);
             PageIt it;
-            it.init(P, pair);
+            it.init(P, &ctrl->w_r0);
             Ring ps{0, 0};
             int u = 0;
             bool ok = true;
@@ -704,7 +795,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
         if (warp == 0 && lane == 0) {  // TMA producer: content columns as two half pages
             prefetch_tensormap(&tm_kv4);
             PageIt it;
-            it.init(P, pair);
+            it.init(P, &ctrl->w_r0);
             Ring vs{0, 0};
             int issued[VH_STAGES];
             uint32_t nph[VH_STAGES] = {};
@@ -738,7 +829,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
         } else if (warp == 1 && lane == 0) {  // MMA issuer: O += P . V
             constexpr uint32_t idesc = idesc_bf16(128, 256, false, true);
             PageIt it;
-            it.init(P, pair);
+            it.init(P, &ctrl->w_r0);
             Ring vs{0, 0}, ps{0, 0};
             uint32_t ncorr = 0, nseg = 0;
             uint32_t vr_ph = 0;  // phase bit of v_ready[i]: it completes only on ragged pages
@@ -814,7 +905,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
             const uint32_t pfree_r = mapa(bar(ctrl->pfree[0]), 0);
             PageIt it;
-            it.init(P, pair);
+            it.init(P, &ctrl->w_r0);
             Ring vs{0, 0}, ps{0, 0}, prev{0, 0};
             int u = 0;
             bool ok = true;
@@ -917,187 +1008,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
-    }
-}
-
-// ---- scheduler: balanced split of all (query row, page) units over the clusters ----------
-__device__ __forceinline__ long long unit_start(int c, long long U, int pairs) {
-    return (long long)c * U / pairs;
-}
-
-constexpr int kSchedSmemRows = 4096;
-__global__ void __launch_bounds__(1024)
-schedule_kernel(int s_q, int rows, const int32_t *__restrict__ seq_lens, int max_seq_len,
-                int max_blocks, int pairs, int32_t *prefix, int32_t *work, int32_t *seg_range,
-                float *m_part, unsigned *err) {
-    __shared__ int warp_tot[32];
-    __shared__ int carry_s;
-    __shared__ int pre_s[kSchedSmemRows + 1];  // the prefix, when it fits (searched below)
-    pdl_trigger();  // the main kernel may start its prologue now
-    const bool in_smem = rows <= kSchedSmemRows;
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    if (tid == 0) carry_s = 0;
-    __syncthreads();
-    for (int base = 0; base < rows; base += 1024) {
-        const int r = base + tid;
-        int n = 0;
-        if (r < rows) {
-            const int b = r / s_q, i = r - b * s_q;
-            const int L = seq_lens[b];
-            if (L < s_q || L > max_seq_len || L > max_blocks * PG) {
-                if (i == 0) record_error(err, kErrBadSeqLen);
-            } else {
-                n = (L - s_q + i + 1 + PG - 1) / PG;
-            }
-        }
-        int x = n;  // inclusive warp scan
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
-        }
-        if (lane == 31) warp_tot[wid] = x;
-        __syncthreads();
-        if (wid == 0) {
-            int t = warp_tot[lane];
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, t, o);
-                if (lane >= o) t += y;
-            }
-            warp_tot[lane] = t;  // inclusive over warps
-        }
-        __syncthreads();
-        const int incl = x + (wid > 0 ? warp_tot[wid - 1] : 0);
-        const int carry = carry_s;
-        if (r < rows) {
-            prefix[r] = carry + incl - n;
-            if (in_smem) pre_s[r] = carry + incl - n;
-        }
-        __syncthreads();
-        if (tid == 1023) carry_s = carry + incl;
-        __syncthreads();
-    }
-    if (tid == 0) {
-        prefix[rows] = carry_s;
-        if (in_smem) pre_s[rows] = carry_s;
-    }
-    // Every partial slot starts empty: a row's slot range also spans clusters that got none of
-    // its pages (when there are fewer pages than clusters), and the combine must skip those.
-    for (size_t i = tid; i < ((size_t)pairs + rows) * NH; i += 1024) m_part[i] = -INFINITY;
-    __syncthreads();
-    const int *pre = in_smem ? pre_s : prefix;
-    const long long U = carry_s;
-    // ---- row-aligned split: every cluster works on one row only, rows get clusters in
-    // proportion to their pages.  A cluster that crosses a row boundary pays a Q reload, a
-    // drain of its pipeline and a second partial write; this split avoids that whenever it is
-    // as balanced as the contiguous one (e.g. every row fits in whole clusters' shares).
-    if (rows <= pairs && rows <= 1024 && in_smem && U > 0) {
-        __shared__ int k_s[1024], cf_s[1025];
-        __shared__ int red_s[32];
-        __shared__ int ok_s, kbase_s, maxload_s;
-        const int r = tid;
-        const int n = r < rows ? pre_s[r + 1] - pre_s[r] : 0;
-        int k = n > 0 ? (int)max(1LL, (long long)n * pairs / U) : 0;
-        // sum of the base counts
-        int x = k;
-        for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-        if (lane == 0) red_s[wid] = x;
-        if (tid == 0) { ok_s = 1; maxload_s = 0; }
-        __syncthreads();
-        if (tid == 0) {
-            int s = 0;
-            for (int i = 0; i < 32; ++i) s += red_s[i];
-            kbase_s = s;
-        }
-        if (r < rows) k_s[r] = k;
-        __syncthreads();
-        const int extra = pairs - kbase_s;
-        if (extra >= 0) {
-            // one more cluster for the `extra` rows with the highest load per cluster (ties: lower row)
-            if (r < rows && n > 0 && extra > 0) {
-                const long long my = (long long)n * 1000000 / k;
-                int rank = 0;
-                for (int i = 0; i < rows; ++i) {
-                    const int ni = pre_s[i + 1] - pre_s[i];
-                    if (ni == 0 || i == r) continue;
-                    const long long li = (long long)ni * 1000000 / k_s[i];
-                    if (li > my || (li == my && i < r)) ++rank;
-                }
-                if (rank < extra) k += 1;
-            }
-            __syncthreads();
-            if (r < rows) {
-                k = min(k, max(n, 0));  // no cluster without pages
-                k_s[r] = k;
-                if (k > 0) atomicMax(&maxload_s, (n + k - 1) / k);
-            }
-            __syncthreads();
-            // accept only if no cluster gets more pages than under the contiguous split: measured
-            // on the uniform batches, a few extra pages cost more than a row change does
-            if (tid == 0) {
-                const long long bal = (U + pairs - 1) / pairs;
-                ok_s = (long long)maxload_s <= bal;
-                int c = 0;
-                for (int i = 0; i < rows; ++i) { cf_s[i] = c; c += k_s[i]; }
-                cf_s[rows] = c;
-            }
-            __syncthreads();
-            if (ok_s) {
-                if (r < rows) {
-                    const int c0 = cf_s[r];
-                    for (int j = 0; j < k; ++j) {
-                        const int p0 = (int)((long long)j * n / k), p1 = (int)((long long)(j + 1) * n / k);
-                        work[4 * (c0 + j) + 0] = r;
-                        work[4 * (c0 + j) + 1] = p0;
-                        work[4 * (c0 + j) + 2] = p1 - p0;
-                        work[4 * (c0 + j) + 3] = 0;
-                    }
-                    seg_range[2 * r] = k > 0 ? c0 + r : 0;
-                    seg_range[2 * r + 1] = k > 0 ? c0 + k + r : 0;
-                }
-                for (int c = cf_s[rows] + tid; c < pairs; c += 1024) {  // idle clusters
-                    work[4 * c + 0] = 0;
-                    work[4 * c + 1] = 0;
-                    work[4 * c + 2] = 0;
-                    work[4 * c + 3] = 0;
-                }
-                return;
-            }
-        }
-    }
-    // ---- contiguous split (any row count)
-    for (int c = tid; c < pairs; c += 1024) {
-        const long long s0 = unit_start(c, U, pairs), s1 = unit_start(c + 1, U, pairs);
-        int r0 = 0;
-        if (s1 > s0) {  // largest r with prefix[r] <= s0
-            int lo = 0, hi = rows - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (pre[mid] <= s0) lo = mid; else hi = mid - 1;
-            }
-            r0 = lo;
-        }
-        work[4 * c + 0] = r0;
-        work[4 * c + 1] = s1 > s0 ? (int)(s0 - pre[r0]) : 0;
-        work[4 * c + 2] = (int)(s1 - s0);
-        work[4 * c + 3] = 0;
-    }
-    for (int r = tid; r < rows; r += 1024) {
-        const long long u0 = pre[r], u1 = pre[r + 1];
-        if (u1 <= u0) {
-            seg_range[2 * r] = 0;
-            seg_range[2 * r + 1] = 0;
-            continue;
-        }
-        auto pair_of = [&](long long u) {
-            int c = (int)(u * pairs / U);
-            while (c + 1 < pairs && unit_start(c + 1, U, pairs) <= u) ++c;
-            while (c > 0 && unit_start(c, U, pairs) > u) --c;
-            return c;
-        };
-        seg_range[2 * r] = pair_of(u0) + r;
-        seg_range[2 * r + 1] = pair_of(u1 - 1) + r + 1;
     }
 }
 
@@ -1220,7 +1130,7 @@ int tc_pairs() {
 struct TcWs {
     uint32_t *o;  // bf16 pairs
     float *m, *l;
-    int32_t *work, *seg_range, *prefix;
+    int32_t *seg_range;
 };
 
 size_t tc_layout(int pairs, int rows, char *base, TcWs *w) {
@@ -1234,16 +1144,12 @@ size_t tc_layout(int pairs, int rows, char *base, TcWs *w) {
     char *o = take(slots * NH * (DC / 2) * sizeof(uint32_t));
     char *m = take(slots * NH * sizeof(float));
     char *l = take(slots * NH * sizeof(float));
-    char *wk = take((size_t)pairs * 4 * sizeof(int32_t));
     char *sr = take((size_t)rows * 2 * sizeof(int32_t));
-    char *pf = take(((size_t)rows + 1) * sizeof(int32_t));
     if (w) {
         w->o = reinterpret_cast<uint32_t *>(o);
         w->m = reinterpret_cast<float *>(m);
         w->l = reinterpret_cast<float *>(l);
-        w->work = reinterpret_cast<int32_t *>(wk);
         w->seg_range = reinterpret_cast<int32_t *>(sr);
-        w->prefix = reinterpret_cast<int32_t *>(pf);
     }
     return off;
 }
@@ -1300,10 +1206,7 @@ cudaError_t launch_decode_tc(const mla_dims_t &d, int B, int s_q, const void *q_
         !tmap_bf16_colblocks(&tm_q9, q_abs, q_rows, ROW, ROW * 2, 64, NCB))
         return cudaErrorInvalidValue;
     unsigned *err = device_error_word();
-    schedule_kernel<<<1, 1024, 0, st>>>(s_q, rows, seq_lens, max_seq_len, max_blocks, pairs, w.prefix,
-                                        w.work, w.seg_range, w.m, err);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
     Params P;
     P.bt = bt;
     P.max_blocks = max_blocks;
@@ -1312,14 +1215,16 @@ cudaError_t launch_decode_tc(const mla_dims_t &d, int B, int s_q, const void *q_
     P.s_q = s_q;
     P.rows = rows;
     P.max_seq_len = max_seq_len;
-    P.work = w.work;
+    P.pairs = pairs;
+    P.seg_range = w.seg_range;
     P.o_part = w.o;
     P.m_part = w.m;
     P.l_part = w.l;
     P.scale_log2 = (float)(1.4426950408889634 / sqrt((double)(d.d_h + d.d_r)));
     P.err = err;
     // The main and combine kernels are launched as programmatic dependents of the kernel before
-    // them: their blocks may start while it drains, and they wait for its results on the device.
+    // them: their blocks may start while it drains, and they wait for its results on the device
+    // before reading any input.
     cudaLaunchAttribute pdl;
     pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl.val.programmaticStreamSerializationAllowed = 1;

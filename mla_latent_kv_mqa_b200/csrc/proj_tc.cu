@@ -173,6 +173,7 @@ __global__ void __launch_bounds__(128, 1)
 absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int n_h, double rope_base,
                  const __nv_bfloat16 *__restrict__ q_c, const __nv_bfloat16 *__restrict__ q_r,
                  const int32_t *__restrict__ pos, __nv_bfloat16 *__restrict__ q_abs, unsigned *err) {
+    pdl_trigger();  // the decode that follows may set itself up (it waits for q_abs on the device)
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_u32(smem_raw);
     const uint32_t data_s = (raw_s + 1023u) & ~1023u;
