@@ -31,7 +31,17 @@
  *              one error word per device (see mla_get_last_device_error) and the scratch
  *              array of mla_decode_fixed_scratch.
  *   Streams    Calls only enqueue work on `stream` (NULL = the legacy default stream)
- *              and return; results are ready in stream order.
+ *              and return; results are ready in stream order.  mla_absorb_q, mla_decode
+ *              and mla_out_proj launch their kernels as programmatic dependents of the
+ *              kernel ahead of them on the stream (CUDA programmatic dependent launch):
+ *              their blocks may start while that kernel drains, and they wait for it on
+ *              the device before reading any activation, cache or table or writing any
+ *              output.
+ *   Weights    w_uk and w_uv are treated as constants of the layer: mla_absorb_q and
+ *              mla_out_proj start reading them before that wait.  Write the weights
+ *              before the first call that uses them and make that write complete
+ *              (synchronize the stream or device, or wait on an event recorded after
+ *              it); do not produce them in the kernel that immediately precedes the call.
  *   Layouts    Row-major, contiguous, as each argument states.
  *   Errors     Arguments are checked on the host before anything is launched; a bad
  *              argument returns an error and launches nothing.  A launch failure
@@ -98,7 +108,8 @@ typedef struct {
  *   pos   [T]             int32 position of each token (>= 0)
  *   w_uk  [n_h*d_h, d_c]  act dtype (the nn.Linear(d_c, n_h*d_h) weight)
  *   q_abs [T, n_h, d_c+d_r] act dtype, written
- * Accumulation is fp32; the rotation angle is formed in fp64.  T == 0 is a no-op.
+ * Accumulation is fp32.  The rotation angle pos * base^(-2k/d_r) is formed in fp64 and reduced
+ * modulo 2 pi in fp64; cos and sin of the reduced angle are fp32.  T == 0 is a no-op.
  * ---------------------------------------------------------------------------------------- */
 mla_status_t mla_absorb_q(const mla_dims_t *dims, int T, const void *q_c, const void *q_r,
                           const int32_t *pos, const void *w_uk, void *q_abs,

@@ -19,11 +19,14 @@ constexpr int kWarpsPerBlock = 8;
 
 template <typename Tin, int KV>  // KV: 0 = f32 cache, 1 = bf16 cache, 2 = fp8 content cache
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
-append_kernel(int T, int d_c, int d_r, int page, double rope_base, const Tin *__restrict__ c_kv,
+append_kernel(int T, int d_c, int d_r, int page, const __grid_constant__ RopeFreqs rope, const Tin *__restrict__ c_kv,
               const Tin *__restrict__ k_r, const int32_t *__restrict__ seq_idx,
               const int32_t *__restrict__ pos, const int32_t *__restrict__ bt, int num_seqs,
               int max_blocks, int num_blocks, void *kv_pool, __nv_bfloat16 *kr_pool,
               float *kv_scale, unsigned *err) {
+    // The query absorption that usually follows may start now: it waits for this kernel on the
+    // device before it reads anything that could depend on it.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
     if (t >= T) return;
@@ -46,7 +49,7 @@ append_kernel(int T, int d_c, int d_r, int page, double rope_base, const Tin *__
     const int half = d_r >> 1;
     for (int k = lane; k < half; k += 32) {
         float cs, sn;
-        rope_cos_sin(k, d_r, rope_base, p, &cs, &sn);
+        rope_cos_sin(rope, k, p, &cs, &sn);
         float x0 = to_f32(k_in[k]), x1 = to_f32(k_in[k + half]);
         float y0 = x0 * cs - x1 * sn;
         float y1 = x1 * cs + x0 * sn;
@@ -95,11 +98,12 @@ cudaError_t launch_append(const mla_dims_t &d, int T, const void *c_kv, const vo
                           void *kr_pool, float *kv_scale, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     dim3 grid((T + kWarpsPerBlock - 1) / kWarpsPerBlock), block(kWarpsPerBlock * 32);
+    const RopeFreqs rope = make_rope_freqs((double)d.rope_base, d.d_r);
     unsigned *err = device_error_word();
     auto *krp = reinterpret_cast<__nv_bfloat16 *>(kr_pool);
 #define MLA_APPEND(TIN, KV)                                                                       \
     append_kernel<TIN, KV><<<grid, block, 0, st>>>(                                                \
-        T, d.d_c, d.d_r, d.page_size, (double)d.rope_base, reinterpret_cast<const TIN *>(c_kv),    \
+        T, d.d_c, d.d_r, d.page_size, rope, reinterpret_cast<const TIN *>(c_kv),    \
         reinterpret_cast<const TIN *>(k_r), seq_idx, pos, bt, num_seqs, max_blocks, num_blocks,    \
         kv_pool, krp, kv_scale, err)
     const bool in_bf16 = d.act_dtype == MLA_DTYPE_BF16;

@@ -209,10 +209,6 @@ __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t a) {
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
     return v;
 }
-__device__ __forceinline__ void st_shared_v4(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
-    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w)
-                 : "memory");
-}
 __device__ __forceinline__ void named_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
@@ -1025,7 +1021,8 @@ combine_tc_kernel(const int32_t *__restrict__ seg_range, const uint32_t *__restr
                   const float *__restrict__ m_part, const float *__restrict__ l_part,
                   float *__restrict__ o_lat, float *__restrict__ lse, int vec_out) {
     const int r = blockIdx.x, cc = blockIdx.y, h = threadIdx.x;
-    pdl_wait();  // the partials of the main kernel
+    pdl_trigger();  // the output projection may start fetching its weights
+    pdl_wait();     // the partials of the main kernel
     const int s0 = seg_range[2 * r], s1 = seg_range[2 * r + 1];
     float M = -INFINITY, L = 0.f, acc[CMB_COLS];
 #pragma unroll

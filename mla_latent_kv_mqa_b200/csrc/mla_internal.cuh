@@ -33,17 +33,34 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
-// RoPE angle tables (구현 section of the MLA article: pair k of a d_r-wide vector is rotated
-// by pos * base^(-2k/d_r)).  The angle is formed and reduced in fp64 so that positions up to
-// 2^31 keep full fp32 accuracy in cos/sin.
-__device__ __forceinline__ void rope_cos_sin(int k, int d_r, double base, int pos, float *c,
-                                             float *s) {
-    double inv_freq = pow(base, -(double)(2 * k) / (double)d_r);
-    double theta = (double)pos * inv_freq;
-    double sd, cd;
-    sincos(theta, &sd, &cd);
-    *c = (float)cd;
-    *s = (float)sd;
+// RoPE angles (구현 section of the MLA article: pair k of a d_r-wide vector is rotated by
+// pos * base^(-2k/d_r)).  The per-pair frequencies are computed once on the host in fp64 and
+// passed by value; on the device the angle pos * f_k is formed in fp64 and reduced to [-pi, pi]
+// by Cody-Waite subtraction of n * 2pi (2pi split into its fp64 value and the remainder, each
+// subtracted with one fused multiply-add), and cos/sin of the reduced angle are taken in fp32.
+// Positions up to 2^31 keep cos/sin within a few fp32 ulps.
+constexpr int kRopeTab = 64;  // pairs held in the table (d_r <= 128); wider d_r computes f_k on the fly
+struct RopeFreqs {
+    double inv_freq[kRopeTab];
+    double base;
+    int d_r;
+};
+inline RopeFreqs make_rope_freqs(double base, int d_r) {
+    RopeFreqs f = {};
+    f.base = base;
+    f.d_r = d_r;
+    for (int k = 0; k < kRopeTab && k < d_r / 2; ++k) f.inv_freq[k] = pow(base, -(double)(2 * k) / (double)d_r);
+    return f;
+}
+__device__ __forceinline__ void rope_cos_sin(const RopeFreqs &f, int k, int pos, float *c, float *s) {
+    constexpr double kTwoPi = 6.283185307179586;        // 2pi rounded to fp64
+    constexpr double kTwoPiRem = 2.4492935982947064e-16;  // 2pi - kTwoPi
+    constexpr double kInvTwoPi = 0.15915494309189535;
+    const double inv = k < kRopeTab ? f.inv_freq[k] : pow(f.base, -(double)(2 * k) / (double)f.d_r);
+    const double theta = (double)pos * inv;
+    const double n = rint(theta * kInvTwoPi);
+    const double r = fma(-n, kTwoPiRem, fma(-n, kTwoPi, theta));
+    sincosf((float)r, s, c);
 }
 
 // Partial results of one split segment, shared by the decode kernels and the combine kernel.

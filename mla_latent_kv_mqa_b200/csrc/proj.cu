@@ -19,7 +19,7 @@ constexpr int kAbsorbTok = 16;    // tokens per block
 // grid (n_h, ceil(d_c/128), ceil(T/16)); block 128.  Thread = one latent column c of head h.
 template <typename Ta>
 __global__ void __launch_bounds__(kAbsorbCols)
-absorb_q_kernel(int T, int n_h, int d_h, int d_c, int d_r, double rope_base,
+absorb_q_kernel(int T, int n_h, int d_h, int d_c, int d_r, const __grid_constant__ RopeFreqs rope,
                 const Ta *__restrict__ q_c, const Ta *__restrict__ q_r,
                 const int32_t *__restrict__ pos, const Ta *__restrict__ w_uk, Ta *__restrict__ q_abs) {
     extern __shared__ float q_s[];  // [kAbsorbTok][d_h]
@@ -54,7 +54,7 @@ absorb_q_kernel(int T, int n_h, int d_h, int d_c, int d_r, double rope_base,
             int tt = i / half, k = i % half;
             int t = t0 + tt;
             float cs, sn;
-            rope_cos_sin(k, d_r, rope_base, pos[t], &cs, &sn);
+            rope_cos_sin(rope, k, pos[t], &cs, &sn);
             const Ta *x = q_r + ((size_t)t * n_h + h) * d_r;
             float x0 = to_f32(x[k]), x1 = to_f32(x[k + half]);
             Ta *y = q_abs + ((size_t)t * n_h + h) * row + d_c;
@@ -104,18 +104,19 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 cudaError_t launch_absorb_q(const mla_dims_t &d, int T, const void *q_c, const void *q_r,
                             const int32_t *pos, const void *w_uk, void *q_abs, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
-    if (!(d.flags & MLA_FLAG_SIMT_PROJ) && proj_tc_supported(d) && aligned16(q_c) && aligned16(w_uk))
+    if (!(d.flags & MLA_FLAG_SIMT_PROJ) && proj_tc_supported(d) && aligned16(q_c) && aligned16(q_r) &&
+        aligned16(w_uk) && aligned16(q_abs))
         return launch_absorb_q_tc(d, T, q_c, q_r, pos, w_uk, q_abs, st);
     dim3 grid(d.n_h, (d.d_c + kAbsorbCols - 1) / kAbsorbCols, (T + kAbsorbTok - 1) / kAbsorbTok);
     size_t smem = sizeof(float) * kAbsorbTok * d.d_h;
     if (d.act_dtype == MLA_DTYPE_BF16) {
         using T_ = __nv_bfloat16;
         absorb_q_kernel<T_><<<grid, kAbsorbCols, smem, st>>>(
-            T, d.n_h, d.d_h, d.d_c, d.d_r, (double)d.rope_base, (const T_ *)q_c, (const T_ *)q_r,
+            T, d.n_h, d.d_h, d.d_c, d.d_r, make_rope_freqs((double)d.rope_base, d.d_r), (const T_ *)q_c, (const T_ *)q_r,
             pos, (const T_ *)w_uk, (T_ *)q_abs);
     } else {
         absorb_q_kernel<float><<<grid, kAbsorbCols, smem, st>>>(
-            T, d.n_h, d.d_h, d.d_c, d.d_r, (double)d.rope_base, (const float *)q_c,
+            T, d.n_h, d.d_h, d.d_c, d.d_r, make_rope_freqs((double)d.rope_base, d.d_r), (const float *)q_c,
             (const float *)q_r, pos, (const float *)w_uk, (float *)q_abs);
     }
     return cudaGetLastError();
