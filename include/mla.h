@@ -151,6 +151,9 @@ size_t mla_decode_workspace_size(const mla_dims_t *dims, int B, int s_q, int max
  *     s_j     = (q_abs[t,h,0:d_c] . c_j + q_abs[t,h,d_c:] . kR_j) / sqrt(d_h + d_r),  j <= P
  *     o_lat   = sum_j softmax(s)_j c_j,       lse = ln sum_j exp(s_j)
  * where (c_j ; kR_j) is cache row j of sequence b (FP8: c_j = e4m3(code) * scale_j).
+ * Precision: bf16 operands, fp32 accumulation and softmax.  With an FP8 cache the kernel
+ * dequantises each page on chip to bf16(e4m3(code) * scale_j), one rounding per value, the
+ * same a bf16 cache applies when it is written.
  * The tokens are split into segments processed in parallel; the partial results are merged
  * exactly by a log-sum-exp combine kernel.
  *   q_abs       [B*s_q, n_h, d_c+d_r] act dtype (from mla_absorb_q)

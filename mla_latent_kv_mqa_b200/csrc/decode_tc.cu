@@ -42,6 +42,7 @@
 // Every wait is bounded (2 s).  On give-up a CTA raises an abort flag in itself and its peer
 // and records MLA_ERR_DEVICE_TIMEOUT; before the teardown every thread that started copies or
 // MMAs waits (again bounded) for them, so no asynchronous write targets a CTA that has left.
+#include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -63,7 +64,6 @@ constexpr int NCB = ROW / 64;               // 9 column blocks per cache row
 // ring stages (heads 0-63, 64-127) through the same box shape over q_abs.
 constexpr int KV_STAGES = 3;
 constexpr int KV_STAGE = NCB * CB;          // 73728
-constexpr int DATA_A = KV_STAGES * KV_STAGE;
 // ---- PV CTA shared memory ----
 constexpr int VH_STAGES = 4;                // ring of half pages: 4 column blocks (256 columns)
 constexpr int VH_STAGE = 4 * CB;            // 32768
@@ -76,9 +76,17 @@ constexpr uint32_t MSG_BYTES = P_TILE + NH * 4 + 4;  // bytes st.async delivers 
 constexpr int P_SLOT = 17408;               // slot stride, 1 KB aligned
 constexpr int P_SLOTS = 3;
 constexpr int DATA_B = P_OFF + P_SLOTS * P_SLOT;
-constexpr int DATA = DATA_A > DATA_B ? DATA_A : DATA_B;
 static_assert(P_SLOT % 1024 == 0 && P_OFF % 1024 == 0 && VH_STAGE % 1024 == 0,
               "swizzled tiles need 1 KB alignment");
+// ---- FP8 cache: e4m3 content codes [page][64][512], a fp32 scale per token, bf16 RoPE keys ----
+// The pages are dequantised on chip, bf16(code * scale), into exactly the bf16 page tiles the
+// bf16 path loads, so everything after the page ring is shared by both.  The codes come in raw
+// (row-major [token][code]) into staging slots: QK CTA whole pages, PV CTA half pages.
+constexpr int STG_CODES = PG * DC;          // 32768: one page's codes
+constexpr int STG_SLOT = 33792;             // codes + 64 scales, 1 KB aligned
+constexpr int VSTG_CODES = PG * DC / 2;     // 16384: codes of one half page ([64][256])
+constexpr int VSTG_SLOT = 17408;
+static_assert(STG_CODES + PG * 4 <= STG_SLOT && VSTG_CODES + PG * 4 <= VSTG_SLOT, "staging slot layout");
 static_assert(MSG_BYTES <= (uint32_t)P_SLOT, "message slot");
 // ---- QK CTA tensor memory: three S buffers, then Q (content and RoPE part) ----
 constexpr uint32_t TMEM_COLS = 512;
@@ -94,11 +102,15 @@ constexpr int SM_THREADS = 256;
 constexpr int SD_WARP0 = 11;                // QK CTA: sender warps 11..14 (P -> CTA 1 by st.async)
 constexpr int SD_THREADS = 128;
 constexpr int EP_WARP0 = 2;                 // PV CTA: correction / epilogue warps 2..5
+constexpr int VC_WARP0 = 6;                 // PV CTA, FP8: converter warps 6..9 (codes -> bf16 V)
+constexpr int VC_THREADS = 128;
 constexpr float RESCALE_LOG2 = 8.0f;
 
 struct __align__(8) Ctrl {
     // QK CTA
     uint64_t kv_full[KV_STAGES], kv_empty[KV_STAGES];
+    uint64_t stg_full[2], stg_empty[2];     // FP8: raw page codes landed / converted
+    uint64_t conv_full[KV_STAGES];          // FP8: a page stage's content columns dequantised
     uint64_t s_full[S_SETS], s_free[S_SETS];
     uint64_t k0_done[S_SETS];   // MMA thread 0 has issued its part of the page in this S buffer
     uint64_t q_ready;
@@ -107,6 +119,7 @@ struct __align__(8) Ctrl {
     // PV CTA
     uint64_t v_full[VH_STAGES], v_empty[VH_STAGES], v_ready[VH_STAGES];
     uint64_t p_full[P_SLOTS], pv_done[P_SLOTS];
+    uint64_t vstg_full[2], vstg_empty[2];   // FP8: raw half-page codes landed / converted
     uint64_t corr_done, o_free;
     uint64_t mma_idle[2];       // drains: one per MMA-issuing thread
     uint32_t tmem_base;
@@ -117,8 +130,20 @@ struct __align__(8) Ctrl {
     float lx[2][NH];            // QK CTA: the second softmax half's row sums, by segment parity
     float fac[2][NH];           // QK CTA: per-head rescale factors of a page, by page parity
 };
-constexpr int SMEM_BYTES = 1024 + DATA + (int)((sizeof(Ctrl) + 127) / 128 * 128);
-static_assert(SMEM_BYTES <= 232448, "shared memory per block");
+// Shared-memory plan of the bf16 (F8 = false) and FP8 (F8 = true) kernels.  The FP8 QK CTA
+// keeps two page stages (its staging slots take the third).
+template <bool F8>
+struct Lay {
+    static constexpr int kv_stages = F8 ? 2 : KV_STAGES;
+    static constexpr int stg_off = kv_stages * KV_STAGE;
+    static constexpr int data_a = stg_off + (F8 ? 2 * STG_SLOT : 0);
+    static constexpr int vstg_off = DATA_B;
+    static constexpr int data_b = DATA_B + (F8 ? 2 * VSTG_SLOT : 0);
+    static constexpr int data = data_a > data_b ? data_a : data_b;
+    static constexpr int smem = 1024 + data + (int)((sizeof(Ctrl) + 127) / 128 * 128);
+};
+static_assert(Lay<false>::smem <= 232448 && Lay<true>::smem <= 232448, "shared memory per block");
+static_assert(Lay<true>::stg_off % 1024 == 0 && Lay<true>::vstg_off % 1024 == 0, "staging alignment");
 
 struct Params {
     const int32_t *bt;
@@ -131,6 +156,8 @@ struct Params {
     float *m_part, *l_part;
     float scale_log2;
     unsigned *err;
+    const uint8_t *codes;     // FP8: content codes [num_blocks][64][512]
+    const float *kv_scale;    // FP8: per-token scales [num_blocks][64]
 };
 
 __device__ __forceinline__ int row_tokens(const Params &P, int r) {
@@ -195,6 +222,28 @@ __device__ __forceinline__ int block_of(const Params &P, int r, int pg) {
         blk = 0;  // keep the copy in bounds; the result is flagged as invalid
     }
     return blk;
+}
+
+// FP8 page tiles: one 8-code group of token row j (codes at src) -> bf16(code * sc), one 16-byte
+// chunk of the K-major SW128 tile at dst.  e4m3 codes are exact in fp16 and fp32, so the code *
+// scale product is rounded once to fp32 and once to bf16.
+// The conversion unit's throughput bounds this (each group costs it 16 instructions).  Variants
+// that build the values with integer and bf16x2 arithmetic instead measured slower in the full
+// kernel.
+__device__ __forceinline__ void dequant8(uint32_t src, float sc, uint32_t dst) {
+    uint32_t w0, w1;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(src));
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t w = (k < 2) ? w0 : w1;
+        const unsigned short pr = (unsigned short)(w >> ((k & 1) * 16));  // codes 2k, 2k+1 (low byte first)
+        uint32_t hh;
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hh) : "h"(pr));
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hh));
+        o[k] = pack_bf16x2(f.x * sc, f.y * sc);
+    }
+    st_shared_v4(dst, o[0], o[1], o[2], o[3]);
 }
 
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
@@ -363,15 +412,22 @@ __device__ __noinline__ void schedule(const Params &P, int pair, uint32_t rank, 
 }
 
 // Named barriers: the 256 softmax threads and the 128 sender threads (QK CTA).
-constexpr int BAR_FAIL = 1, BAR_Q = 2, BAR_SFAIL = 3, BAR_SFLAG = 4;
+constexpr int BAR_FAIL = 1, BAR_Q = 2, BAR_SFAIL = 3, BAR_SFLAG = 4, BAR_CONV = 5;
+constexpr int BAR_VCONV = 5;  // PV CTA: the FP8 converter warps
 
+// F8 = false: bf16 cache; tm_kv9 loads whole pages {64, 64, 9}, tm_kv4 half pages {64, 64, 4}.
+// F8 = true: FP8 cache; tm_kv9 loads a page's RoPE keys as one {64, 64} tile, tm_kv4 a half
+// page of raw codes {256, 64}; the codes of whole pages and the scales come by bulk copy.
+template <bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_constant__ CUtensorMap tm_kv4,
                  const __grid_constant__ CUtensorMap tm_q9, const __grid_constant__ Params P) {
+    using L = Lay<F8>;
+    constexpr int KVS = L::kv_stages;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_u32(smem_raw);
     const uint32_t data_s = (raw_s + 1023u) & ~1023u;
-    Ctrl *ctrl = reinterpret_cast<Ctrl *>(smem_raw + (data_s - raw_s) + DATA);
+    Ctrl *ctrl = reinterpret_cast<Ctrl *>(smem_raw + (data_s - raw_s) + L::data);
     volatile uint32_t *abort_flag = &ctrl->abort;
     auto bar = [&](uint64_t &b) { return smem_u32(&b); };
 
@@ -386,6 +442,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
         for (int i = 0; i < KV_STAGES; ++i) {
             mbar_init(bar(ctrl->kv_full[i]), 1);
             mbar_init(bar(ctrl->kv_empty[i]), 2);  // both MMA threads (or the Q copy, twice)
+            mbar_init(bar(ctrl->conv_full[i]), SM_THREADS / 32);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(ctrl->stg_full[i]), 1);
+            mbar_init(bar(ctrl->stg_empty[i]), SM_THREADS / 32);
+            mbar_init(bar(ctrl->vstg_full[i]), 1);
+            mbar_init(bar(ctrl->vstg_empty[i]), VC_THREADS / 32);
         }
         for (int i = 0; i < S_SETS; ++i) {
             mbar_init(bar(ctrl->s_full[i]), 2);
@@ -401,7 +464,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             mbar_init(bar(ctrl->pv_done[i]), 1);
         }
         for (int i = 0; i < VH_STAGES; ++i) {
-            mbar_init(bar(ctrl->v_full[i]), 1);
+            mbar_init(bar(ctrl->v_full[i]), F8 ? VC_THREADS / 32 : 1);  // TMA, or the FP8 converters
             mbar_init(bar(ctrl->v_empty[i]), 1);
             mbar_init(bar(ctrl->v_ready[i]), 4);
         }
@@ -462,7 +525,29 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 PROF_MARK(1);
                 issued[st.i] = 1;
                 nph[st.i] = st.ph;
-                st.adv(KV_STAGES);
+                st.adv(KVS);
+                return true;
+            };
+            // FP8: a page's raw codes and scales go to a staging slot (the softmax warps dequantise
+            // them into the page stage); its RoPE keys go straight to the stage's last column block.
+            Ring g{0, 0};
+            int g_issued[2] = {0, 0};
+            uint32_t g_nph[2] = {0u, 0u};
+            auto load_f8 = [&](int blk) -> bool {
+                if (!wait(bar(ctrl->stg_empty[g.i]), g.ph ^ 1u, abort_flag)) return false;
+                const uint32_t sdst = data_s + L::stg_off + g.i * STG_SLOT;
+                mbar_arrive_expect_tx(bar(ctrl->stg_full[g.i]), STG_CODES + PG * 4);
+                bulk_load(sdst, P.codes + (size_t)blk * STG_CODES, STG_CODES, bar(ctrl->stg_full[g.i]));
+                bulk_load(sdst + STG_CODES, P.kv_scale + (size_t)blk * PG, PG * 4, bar(ctrl->stg_full[g.i]));
+                g_issued[g.i] = 1;
+                g_nph[g.i] = g.ph;
+                g.adv(2);
+                if (!wait(bar(ctrl->kv_empty[st.i]), st.ph ^ 1u, abort_flag)) return false;
+                mbar_arrive_expect_tx(bar(ctrl->kv_full[st.i]), CB);
+                tma_load_2d(data_s + st.i * KV_STAGE + (NCB - 1) * CB, &tm_kv9, 0, blk * PG, bar(ctrl->kv_full[st.i]));
+                issued[st.i] = 1;
+                nph[st.i] = st.ph;
+                st.adv(KVS);
                 return true;
             };
             while (ok && !it.done()) {
@@ -470,7 +555,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                     if (!(ok = load(&tm_q9, it.r * NH) && load(&tm_q9, it.r * NH + 64))) break;
                     TRACE(1, u);
                 }
-                if (!(ok = load(&tm_kv9, block_of(P, it.r, it.pg) * PG))) break;
+                const int blk = block_of(P, it.r, it.pg);
+                if (!(ok = F8 ? load_f8(blk) : load(&tm_kv9, blk * PG))) break;
                 PROF_PAGE();
                 TRACE(2, u);
                 ++u;
@@ -480,6 +566,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             PROF_FLUSH();
             for (int i = 0; i < KV_STAGES; ++i)  // drain: every copy this thread started has landed
                 if (issued[i]) wait(bar(ctrl->kv_full[i]), nph[i], never);
+            for (int i = 0; i < 2; ++i)
+                if (g_issued[i]) wait(bar(ctrl->stg_full[i]), g_nph[i], never);
         } else if ((warp == 1 || warp == 2) && lane == 0) {  // MMA issuers: S += Q . KV^T, split K
             // Both threads work on every page: thread 0 column blocks 0-4, thread 1 blocks 5-8 (the
             // RoPE part).  One thread cannot issue N = 64 MMAs as fast as the tensor core runs them,
@@ -497,12 +585,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             it.init(P, &ctrl->w_r0);
             Ring st{0, 0}, sb{0, 0};
             uint32_t qn = 0;
+            uint32_t cv_ph = 0;  // FP8: phase bit of conv_full[i] (it completes on page uses only)
             int u = 0;
             bool ok = true, any = false;
             PROF_DECL
             while (ok && !it.done()) {
                 if (it.first) {
-                    st.adv(KV_STAGES, 2);  // the segment's Q stages (copied to TMEM by the softmax warps)
+                    st.adv(KVS, 2);  // the segment's Q stages (copied to TMEM by the softmax warps)
                     PROF_MARK(4);
                     if (!(ok = wait(bar(ctrl->q_ready), qn & 1u, abort_flag))) break;
                     PROF_MARK(0);
@@ -516,6 +605,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 // TMA-filled shared memory needs no tcgen05 fence: the mbarrier completion already
                 // makes it visible to MMAs issued after the wait.
                 if (!(ok = wait(bar(ctrl->kv_full[st.i]), st.ph, abort_flag))) break;
+                if (F8) {  // the content columns are written by the softmax warps' dequantisation
+                    if (!(ok = wait(bar(ctrl->conv_full[st.i]), (cv_ph >> st.i) & 1u, abort_flag))) break;
+                    cv_ph ^= 1u << st.i;
+                }
                 PROF_MARK(2);
                 TRACE(6 + part, u);
                 const uint32_t d = tmem + S_COL + sb.i * PG;
@@ -538,7 +631,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 any = true;
                 TRACE(3 + part, u);
                 ++u;
-                st.adv(KV_STAGES);
+                st.adv(KVS);
                 sb.adv(S_SETS);
                 it.next(P);
             }
@@ -565,9 +658,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             // column blocks 0-4 (half 0) or 5-8 (half 1).  Uniform across the 256 threads.
             auto load_q = [&]() -> bool {
                 const Ring q0 = st;
-                st.adv(KV_STAGES);
+                st.adv(KVS);
                 const Ring q1 = st;
-                st.adv(KV_STAGES);
+                st.adv(KVS);
                 const bool w = wait(bar(ctrl->kv_full[q0.i]), q0.ph, abort_flag) &&
                                wait(bar(ctrl->kv_full[q1.i]), q1.ph, abort_flag);
                 if (named_red_or(!w, BAR_Q, SM_THREADS)) return false;
@@ -600,6 +693,34 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 return true;
             };
 
+            // FP8: dequantise the page whose raw codes are in staging slot cg into page stage c
+            // (sixteen 8-code groups per thread), then release the slot and report the stage.
+            // Pages are converted one ahead of the softmax: the next page of the segment before
+            // this page's softmax, a segment's first page right after its Q copy.
+            Ring cg{0, 0};
+            auto convert = [&](Ring c) -> bool {
+                const bool w = wait(bar(ctrl->stg_full[cg.i]), cg.ph, abort_flag) &&
+                               wait(bar(ctrl->kv_empty[c.i]), c.ph ^ 1u, abort_flag);
+                if (named_red_or(!w, BAR_CONV, SM_THREADS)) return false;
+                const uint32_t src = data_s + L::stg_off + cg.i * STG_SLOT;
+                const float *scl = reinterpret_cast<const float *>(smem_raw + (src - raw_s) + STG_CODES);
+                const uint32_t dst = data_s + c.i * KV_STAGE;
+#pragma unroll 4
+                for (int q = t; q < PG * (DC / 8); q += SM_THREADS) {  // 4096 groups, 16 per thread
+                    const int j = q >> 6, cc = q & 63;
+                    dequant8(src + j * DC + cc * 8, scl[j], dst + (cc >> 3) * CB + j * 128 + (((cc & 7) ^ (j & 7)) << 4));
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(bar(ctrl->conv_full[c.i]));
+                    mbar_arrive(bar(ctrl->stg_empty[cg.i]));
+                }
+                cg.adv(2);
+                return true;
+            };
+            auto first_page = [&]() -> bool { return !F8 || convert(st); };
+
             {   // the MMAs only accumulate into S: start from zero
                 uint32_t z[32];
 #pragma unroll
@@ -607,9 +728,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 for (int i = 0; i < S_SETS; ++i) tmem_st32(tmem + lane_base + S_COL + i * PG + half * 32, z);
                 tmem_wait_st();
             }
-            if (!it.done()) ok = load_q();  // its barrier also orders the zeroing before q_ready
+            if (!it.done()) ok = load_q() && first_page();  // load_q's barrier also orders the zeroing before q_ready
             PROF_DECL
             while (ok && !it.done()) {
+                if (F8 && !it.last()) {  // the next page of this segment (its stage follows this page's)
+                    Ring c = st;
+                    c.adv(KVS);
+                    if (!(ok = convert(c))) break;
+                    PROF_MARK(6);
+                }
                 if (t == 0) TRACE(27, u);
                 if (t == 32) TRACE(67, u);
                 bool good = wait(bar(ctrl->s_full[sb.i]), sb.ph, abort_flag);
@@ -637,7 +764,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 if (t == 0) TRACE(24, u);
                 if (t == 32) TRACE(64, u);
                 sb.adv(S_SETS);
-                st.adv(KV_STAGES);  // this page's stage
+                st.adv(KVS);  // this page's stage
 
                 const bool first = it.first, last = it.last();
                 const int valid = it.valid();
@@ -718,7 +845,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                     ++seg;
                     // The last page's S is complete, so every QK MMA of this segment has finished
                     // and the next segment's Q may overwrite TMEM now.
-                    if (it.left > 1 && !(ok = load_q())) break;
+                    if (it.left > 1 && !(ok = load_q() && first_page())) break;
                     PROF_MARK(6);
                 }
                 it.next(P);
@@ -799,9 +926,22 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             int u = 0;
             bool ok = true;
             PROF_DECL
+            Ring vg{0, 0};  // FP8: staging slot of the next half page of raw codes
+            int g_issued[2] = {0, 0};
+            uint32_t g_nph[2] = {0u, 0u};
             while (ok && !it.done()) {
                 const int blk = block_of(P, it.r, it.pg);
-                for (int hh = 0; hh < 2; ++hh) {
+                for (int hh = 0; F8 && hh < 2; ++hh) {  // FP8: codes [64][256] + scales -> staging
+                    if (!(ok = wait(bar(ctrl->vstg_empty[vg.i]), vg.ph ^ 1u, abort_flag))) break;
+                    const uint32_t sdst = data_s + L::vstg_off + vg.i * VSTG_SLOT;
+                    mbar_arrive_expect_tx(bar(ctrl->vstg_full[vg.i]), VSTG_CODES + PG * 4);
+                    tma_load_2d(sdst, &tm_kv4, hh * (DC / 2), blk * PG, bar(ctrl->vstg_full[vg.i]));
+                    bulk_load(sdst + VSTG_CODES, P.kv_scale + (size_t)blk * PG, PG * 4, bar(ctrl->vstg_full[vg.i]));
+                    g_issued[vg.i] = 1;
+                    g_nph[vg.i] = vg.ph;
+                    vg.adv(2);
+                }
+                for (int hh = 0; !F8 && hh < 2; ++hh) {
                     PROF_MARK(1);
                     if (!(ok = wait(bar(ctrl->v_empty[vs.i]), vs.ph ^ 1u, abort_flag))) break;
                     PROF_MARK(0);
@@ -822,6 +962,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             PROF_FLUSH();
             for (int i = 0; i < VH_STAGES; ++i)
                 if (issued[i]) wait(bar(ctrl->v_full[i]), nph[i], never);
+            for (int i = 0; i < 2; ++i)
+                if (g_issued[i]) wait(bar(ctrl->vstg_full[i]), g_nph[i], never);
         } else if (warp == 1 && lane == 0) {  // MMA issuer: O += P . V
             constexpr uint32_t idesc = idesc_bf16(128, 256, false, true);
             PageIt it;
@@ -895,6 +1037,47 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                     wait<true>(bar(ctrl->p_full[ps.i]), ps.ph, never, 1000000ull);
                     ps.adv(P_SLOTS);
                 }
+        } else if (F8 && warp >= VC_WARP0 && warp < VC_WARP0 + 4) {  // FP8: codes -> bf16 V stages
+            const int t = threadIdx.x - VC_WARP0 * 32;  // 0..127
+            PageIt it;
+            it.init(P, &ctrl->w_r0);
+            Ring vs{0, 0}, vg{0, 0};
+            bool ok = true;
+            PROF_DECL
+            while (ok && !it.done()) {
+                for (int hh = 0; hh < 2; ++hh) {
+                    bool w = wait(bar(ctrl->vstg_full[vg.i]), vg.ph, abort_flag);
+                    PROF_MARK(0);
+                    w = w && wait(bar(ctrl->v_empty[vs.i]), vs.ph ^ 1u, abort_flag);
+                    PROF_MARK(1);
+                    if (named_red_or(!w, BAR_VCONV, VC_THREADS)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t src = data_s + L::vstg_off + vg.i * VSTG_SLOT;
+                    const float *scl = reinterpret_cast<const float *>(smem_raw + (src - raw_s) + VSTG_CODES);
+                    const uint32_t dst = data_s + V_OFF + vs.i * VH_STAGE;
+#pragma unroll 4
+                    for (int q = t; q < PG * (DC / 16); q += VC_THREADS) {  // 64 tokens x 32 groups
+                        const int j = q >> 5, cc = q & 31;
+                        dequant8(src + j * (DC / 2) + cc * 8, scl[j],
+                                 dst + (cc >> 3) * CB + j * 128 + (((cc & 7) ^ (j & 7)) << 4));
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(bar(ctrl->v_full[vs.i]));
+                        mbar_arrive(bar(ctrl->vstg_empty[vg.i]));
+                    }
+                    PROF_MARK(2);
+                    vs.adv(VH_STAGES);
+                    vg.adv(2);
+                }
+                PROF_PAGE();
+                it.next(P);
+            }
+            if (!ok && lane == 0) fail();
+            PROF_FLUSH();
         } else if (warp >= EP_WARP0 && warp < EP_WARP0 + 4) {  // ragged zeroing, rescale, epilogue
             const int quarter = warp & 3;
             const int h = quarter * 32 + lane;
@@ -1093,13 +1276,15 @@ combine_tc_kernel(const int32_t *__restrict__ seg_range, const uint32_t *__restr
 }
 
 // ---- host side ------------------------------------------------------------------------------
-int g_pairs[64] = {};
+int g_pairs[2][64] = {};
 
+// Co-resident clusters of the kernel on the current device (cached per device).
+template <bool F8>
 int tc_pairs() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    if (g_pairs[dev]) return g_pairs[dev];
-    if (cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+    if (g_pairs[F8][dev]) return g_pairs[F8][dev];
+    if (cudaFuncSetAttribute(decode_tc_kernel<F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay<F8>::smem) !=
         cudaSuccess)
         return 0;
     int sms = 148;
@@ -1107,7 +1292,7 @@ int tc_pairs() {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (sms / 2));
     cfg.blockDim = dim3(THREADS);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.dynamicSmemBytes = Lay<F8>::smem;
     cudaLaunchAttribute attr;
     attr.id = cudaLaunchAttributeClusterDimension;
     attr.val.clusterDim.x = 2;
@@ -1116,12 +1301,15 @@ int tc_pairs() {
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, decode_tc_kernel, &cfg) != cudaSuccess || n < 1) {
+    if (cudaOccupancyMaxActiveClusters(&n, decode_tc_kernel<F8>, &cfg) != cudaSuccess || n < 1) {
         cudaGetLastError();
         n = sms / 2;
     }
-    g_pairs[dev] = n;
+    g_pairs[F8][dev] = n;
     return n;
+}
+int tc_pairs(const mla_dims_t &d) {
+    return d.kv_dtype == MLA_DTYPE_FP8_E4M3 ? tc_pairs<true>() : tc_pairs<false>();
 }
 
 struct TcWs {
@@ -1178,30 +1366,33 @@ extern "C" int mla_prof_dump(unsigned long long *host) {
 
 bool tc_supported(const mla_dims_t &d) {
     return d.n_h == NH && d.d_c == DC && d.d_r == ROW - DC && d.page_size == PG &&
-           d.act_dtype == MLA_DTYPE_BF16 && d.kv_dtype == MLA_DTYPE_BF16;
+           d.act_dtype == MLA_DTYPE_BF16 && (d.kv_dtype == MLA_DTYPE_BF16 || d.kv_dtype == MLA_DTYPE_FP8_E4M3);
 }
 
-size_t tc_workspace_bytes(const mla_dims_t &, int B, int s_q, int) {
-    const int pairs = tc_pairs();
+size_t tc_workspace_bytes(const mla_dims_t &d, int B, int s_q, int) {
+    const int pairs = tc_pairs(d);
     if (pairs < 1) return 0;
     return tc_layout(pairs, B * s_q, nullptr, nullptr);
 }
 
 cudaError_t launch_decode_tc(const mla_dims_t &d, int B, int s_q, const void *q_abs,
-                             const void *kv_pool, const void *, const float *, const int32_t *bt,
+                             const void *kv_pool, const void *kr_pool, const float *kv_scale, const int32_t *bt,
                              int max_blocks, int num_blocks, const int32_t *seq_lens, int max_seq_len,
                              void *ws, size_t ws_bytes, float *o_lat, float *lse, cudaStream_t st) {
     const int rows = B * s_q;
-    const int pairs = tc_pairs();
+    const bool f8 = d.kv_dtype == MLA_DTYPE_FP8_E4M3;
+    const int pairs = tc_pairs(d);
     if (pairs < 1) return cudaErrorNotSupported;
     TcWs w;
     if (tc_layout(pairs, rows, reinterpret_cast<char *>(ws), &w) > ws_bytes) return cudaErrorInvalidValue;
     CUtensorMap tm_kv9, tm_kv4, tm_q9;
     const uint64_t pool_rows = (uint64_t)num_blocks * PG, q_rows = (uint64_t)rows * NH;
-    if (!tmap_bf16_colblocks(&tm_kv9, kv_pool, pool_rows, ROW, ROW * 2, PG, NCB) ||
-        !tmap_bf16_colblocks(&tm_kv4, kv_pool, pool_rows, ROW, ROW * 2, PG, 4) ||
-        !tmap_bf16_colblocks(&tm_q9, q_abs, q_rows, ROW, ROW * 2, 64, NCB))
-        return cudaErrorInvalidValue;
+    const bool maps =
+        f8 ? (tmap_bf16_2d(&tm_kv9, kr_pool, ROW - DC, pool_rows, (ROW - DC) * 2, 64, PG) &&
+              tmap_u8_rows(&tm_kv4, kv_pool, DC, pool_rows, DC, DC / 2, PG))
+           : (tmap_bf16_colblocks(&tm_kv9, kv_pool, pool_rows, ROW, ROW * 2, PG, NCB) &&
+              tmap_bf16_colblocks(&tm_kv4, kv_pool, pool_rows, ROW, ROW * 2, PG, 4));
+    if (!maps || !tmap_bf16_colblocks(&tm_q9, q_abs, q_rows, ROW, ROW * 2, 64, NCB)) return cudaErrorInvalidValue;
     unsigned *err = device_error_word();
     cudaError_t e;
     Params P;
@@ -1219,6 +1410,8 @@ cudaError_t launch_decode_tc(const mla_dims_t &d, int B, int s_q, const void *q_
     P.l_part = w.l;
     P.scale_log2 = (float)(1.4426950408889634 / sqrt((double)(d.d_h + d.d_r)));
     P.err = err;
+    P.codes = f8 ? reinterpret_cast<const uint8_t *>(kv_pool) : nullptr;
+    P.kv_scale = f8 ? kv_scale : nullptr;
     // The main and combine kernels are launched as programmatic dependents of the kernel before
     // them: their blocks may start while it drains, and they wait for its results on the device
     // before reading any input.
@@ -1228,7 +1421,7 @@ cudaError_t launch_decode_tc(const mla_dims_t &d, int B, int s_q, const void *q_
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs);
     cfg.blockDim = dim3(THREADS);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.dynamicSmemBytes = f8 ? Lay<true>::smem : Lay<false>::smem;
     cfg.stream = st;
     cfg.attrs = &pdl;
 #ifdef MLA_NO_PDL
@@ -1236,7 +1429,8 @@ cudaError_t launch_decode_tc(const mla_dims_t &d, int B, int s_q, const void *q_
 #else
     cfg.numAttrs = 1;
 #endif
-    e = cudaLaunchKernelEx(&cfg, decode_tc_kernel, tm_kv9, tm_kv4, tm_q9, P);
+    e = f8 ? cudaLaunchKernelEx(&cfg, decode_tc_kernel<true>, tm_kv9, tm_kv4, tm_q9, P)
+           : cudaLaunchKernelEx(&cfg, decode_tc_kernel<false>, tm_kv9, tm_kv4, tm_q9, P);
     if (e != cudaSuccess) return e;
     const int vec_out = (reinterpret_cast<uintptr_t>(o_lat) & 15) == 0;
     cfg.gridDim = dim3(rows, DC / CMB_COLS);

@@ -171,6 +171,13 @@ __device__ __forceinline__ void bulk_wait_group_read_le1() {
     asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait_group_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Untiled bulk copy global -> this CTA's shared memory, completing on `bar` (16-byte aligned
+// addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
 // Per-thread 16-byte global -> shared copy (L2 only), completed by cp_async_wait_all(), after
 // which the issuing thread sees the bytes.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {

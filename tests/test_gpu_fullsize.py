@@ -1,5 +1,5 @@
 """Parity at the full workload sizes, in the launch configuration bench.py times (the default
-path of mla_decode: tensor cores for the bf16 cache, CUDA cores for the FP8 cache).
+path of mla_decode: the tensor-core kernel, for the bf16 and the FP8 cache).
 
 The whole decode step runs on the GPU for every query row.  The fp64 oracle is run on a seeded
 sample of sequences and heads that it computes in seconds; the tolerances are those of

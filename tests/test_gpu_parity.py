@@ -44,6 +44,8 @@ SMALL = {
     "v3_permuted": dict(seed=22, seq_lens=[700, 33, 1000, 64 * 5], permute=True, spare=8),
     "v3_lognormal": dict(seed=23, seq_lens=[3000], lognormal_tokens=True),
     "fp8_sq2": dict(seed=24, seq_lens=[300, 2, 65, 128], s_q=2, kv_dtype="fp8"),
+    "fp8_ragged_permuted": dict(seed=27, seq_lens=[200, 64, 1, 129, 700], kv_dtype="fp8", permute=True, spare=4),
+    "fp8_lognormal": dict(seed=28, seq_lens=[2000], lognormal_tokens=True, kv_dtype="fp8"),
     "bf16_sq2": dict(seed=25, seq_lens=[513, 3], s_q=2),
     # more query rows than the tensor-core kernel has clusters: the scheduler's contiguous split
     "many_rows": dict(seed=26, seq_lens=[int(x) for x in np.random.default_rng(26).integers(1, 300, 96)]),
