@@ -39,6 +39,11 @@ WORKLOADS = {
     "mtp_fp8": "V3 dims, batch 128, context 8192, s_q=2 causal, FP8 e4m3 content + bf16 RoPE key",
 }
 FLUSH_BYTES = 512 << 20
+# DRAM bytes (read + write) per launch of the main decode kernel, from one ncu capture of the
+# same workload and build (`ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum -k
+# regex:decode_tc_kernel -s 2 -c 1 python bench.py --plain-steps 3 --batch 16`, caches flushed
+# before the launch as in the timed loop).  None where no capture of that workload exists.
+DECODE_TRAFFIC = {"v3": 78050048 + 2524160}
 
 
 def make_workload(name: str, batch: int | None = None):
@@ -50,7 +55,7 @@ def make_workload(name: str, batch: int | None = None):
     if name == "long":
         return W.long_decode()
     if name == "mtp_fp8":
-        return W.mtp_fp8_decode()
+        return W.mtp_fp8_decode(B=batch or 128)
     raise SystemExit(f"unknown config {name}")
 
 
@@ -355,7 +360,7 @@ def run_mine(args):
                    "frac_hbm": gbs / hbm_peak, "frac_bf16": tfl / tc_peak,
                    "cache_bytes": cache_bytes, "flops": flops},
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak, "traffic": None, "peak_source": src,
+                     "frac": achieved / peak, "traffic": DECODE_TRAFFIC.get(args.config), "peak_source": src,
                      "kernel": "mla_decode", "algorithmic_per_launch": cache_bytes if bound == "hbm" else flops},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
@@ -372,8 +377,8 @@ def run_mine(args):
 
 def run_plain(args):
     """--plain-steps N: N eager (non-graph, untimed) steps of the workload, then exit 0.  The
-    command profilers (ncu) are pointed at; --batch overrides the v3 batch, e.g. 32 so that the
-    cache (151 MB) exceeds the 126 MB L2."""
+    command profilers (ncu) are pointed at; --batch overrides the batch of v3 (e.g. 32, so that
+    the 151 MB cache exceeds the 126 MB L2) or of mtp_fp8."""
     import torch
     from tests.harness import GpuRun
     wl = make_workload(args.config, args.batch)
@@ -395,7 +400,7 @@ def main():
     ap.add_argument("--config", default="v3", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--plain-steps", type=int, default=0, help="run N untimed eager steps and exit (profiling)")
-    ap.add_argument("--batch", type=int, default=None, help="with --plain-steps: batch of the v3 workload")
+    ap.add_argument("--batch", type=int, default=None, help="with --plain-steps: batch of the v3 or mtp_fp8 workload")
     args = ap.parse_args()
     if args.plain_steps:
         run_plain(args)

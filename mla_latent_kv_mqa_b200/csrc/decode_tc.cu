@@ -227,9 +227,8 @@ __device__ __forceinline__ int block_of(const Params &P, int r, int pg) {
 // FP8 page tiles: one 8-code group of token row j (codes at src) -> bf16(code * sc), one 16-byte
 // chunk of the K-major SW128 tile at dst.  e4m3 codes are exact in fp16 and fp32, so the code *
 // scale product is rounded once to fp32 and once to bf16.
-// The conversion unit's throughput bounds this (each group costs it 16 instructions).  Variants
-// that build the values with integer and bf16x2 arithmetic instead measured slower in the full
-// kernel.
+// Each group costs 16 conversion instructions.  Variants that build the values with integer and
+// bf16x2 arithmetic instead (exact as well) measured slower in the full kernel.
 __device__ __forceinline__ void dequant8(uint32_t src, float sc, uint32_t dst) {
     uint32_t w0, w1;
     asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(src));
@@ -307,6 +306,16 @@ __device__ __forceinline__ void trace_event(int pair, uint32_t code, uint32_t un
 #define TRACE(code, unit) trace_event(pair, (code), (uint32_t)(unit), tr_n)
 #else
 #define TRACE(code, unit) ((void)0)
+#endif
+
+#ifdef MLA_SPAN
+// Development instrumentation: globaltimer stamps of the phases of every CTA of the last launch
+// (0 entry, 1 set up, 2 dependency wait done, 3 scheduled, 4 first S read, 5 last softmax done,
+// 6 last epilogue done, 7 exit).
+__device__ unsigned long long g_span[512][8];
+#define SPAN(i) (g_span[blockIdx.x & 511][i] = globaltimer())
+#else
+#define SPAN(i) ((void)0)
 #endif
 
 #ifdef MLA_PROF
@@ -411,6 +420,20 @@ __device__ __noinline__ void schedule(const Params &P, int pair, uint32_t rank, 
     __syncthreads();
 }
 
+// Warms L2 (and the address translation) for the sequence lengths and the block table, which
+// the schedule and the first page loads read through a chain of dependent accesses.  A prefetch
+// returns nothing and L2 is coherent, so it may precede the wait for the kernel before this one.
+__device__ __noinline__ void warm_tables(const Params &P) {
+    const int nb = P.rows / P.s_q;
+    const char *sl = reinterpret_cast<const char *>(P.seq_lens);
+    for (int off = threadIdx.x * 128; off < nb * 4; off += THREADS * 128) prefetch_l2(sl + off);
+    const char *btp = reinterpret_cast<const char *>(P.bt);
+    const size_t bt_bytes = (size_t)nb * P.max_blocks * 4;
+    for (size_t off = ((size_t)blockIdx.x * THREADS + threadIdx.x) * 128; off < bt_bytes;
+         off += (size_t)gridDim.x * THREADS * 128)
+        prefetch_l2(btp + off);
+}
+
 // Named barriers: the 256 softmax threads and the 128 sender threads (QK CTA).
 constexpr int BAR_FAIL = 1, BAR_Q = 2, BAR_SFAIL = 3, BAR_SFLAG = 4, BAR_CONV = 5;
 constexpr int BAR_VCONV = 5;  // PV CTA: the FP8 converter warps
@@ -434,6 +457,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
     const uint32_t rank = cluster_ctarank();
     const int pair = blockIdx.x >> 1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) SPAN(0);
+    warm_tables(P);
 #ifdef MLA_TRACE
     uint32_t tr_n = 0;
 #endif
@@ -486,10 +511,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
     __syncthreads();
     tc_fence_after();
     cluster_sync();
+    if (threadIdx.x == 0) SPAN(1);
     // Everything above overlaps the kernel before this one; inputs are read from here on.
     pdl_trigger();
     pdl_wait();
+    if (threadIdx.x == 0) SPAN(2);
     schedule(P, pair, rank, ctrl);
+    if (threadIdx.x == 0) SPAN(3);
     const uint32_t tmem = ctrl->tmem_base;
     const uint32_t peer = rank ^ 1u;
     if (threadIdx.x == 0) TRACE(20 + rank, (uint32_t)clock64() >> 8);
@@ -740,6 +768,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 if (t == 0) TRACE(27, u);
                 if (t == 32) TRACE(67, u);
                 bool good = wait(bar(ctrl->s_full[sb.i]), sb.ph, abort_flag);
+                if (t == 0 && u == 0) SPAN(4);
                 PROF_MARK(0);
                 if (t == 0) TRACE(5, u);
                 if (t == 32) TRACE(45, u);
@@ -851,6 +880,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 it.next(P);
             }
             if (!ok) fail();
+            if (t == 0) SPAN(5);
             PROF_FLUSH();
         } else if (warp >= SD_WARP0 && warp < SD_WARP0 + 4) {  // senders: P in TMEM -> CTA 1 slot
             const int t = threadIdx.x - SD_WARP0 * 32;          // 0..127
@@ -1164,6 +1194,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(ctrl->o_free));
                     if (h == 0) TRACE(19, u);
+                    if (h == 0) SPAN(6);
                 }
                 PROF_MARK(3);
                 PROF_PAGE();
@@ -1181,6 +1212,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
     // ---- teardown: both CTAs quiesce before either releases TMEM or exits ----
     __syncwarp();
     if (threadIdx.x == 0) TRACE(22 + rank, (uint32_t)clock64() >> 8);
+    if (threadIdx.x == 0) SPAN(7);
     tc_fence_before();
     __syncthreads();
     cluster_sync();
@@ -1350,6 +1382,15 @@ extern "C" int mla_trace_dump(uint32_t *host, int max_entries) {
     static uint32_t zeros[2 * kTraceMax];
     cudaMemcpyToSymbol(g_trace, zeros, sizeof(zeros));
     return n;
+}
+#endif
+
+#ifdef MLA_SPAN
+// Copies the phase stamps (512 x 8 u64) of the last launch.
+extern "C" int mla_span_dump(unsigned long long *host) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+    cudaMemcpyFromSymbol(host, g_span, sizeof(g_span));
+    return 0;
 }
 #endif
 

@@ -193,6 +193,10 @@ __device__ __forceinline__ void ld_shared_f4(uint32_t a, float *x) {
                  : "r"(a)
                  : "memory");
 }
+// Hint: bring the 128-byte line at p into L2 (no result, no architectural read).
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
