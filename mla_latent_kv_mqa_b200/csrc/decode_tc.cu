@@ -1,5 +1,5 @@
 // Tensor-core (tcgen05 / TMEM / TMA) absorbed-MLA decode for the DeepSeek-V3 shape
-// (n_h = 128, d_c = 512, d_R = 64, 64-token pages, bf16 cache).
+// (n_h = 128, d_c = 512, d_R = 64, 64-token pages), bf16 or FP8 cache.
 //
 // What it computes -- MLA article (itwiki "멀티 헤드 잠재 어텐션"), section 분리 RoPE output
 // equation in the absorbed form of section 행렬 흡수: for query row t and head h,
@@ -30,6 +30,12 @@
 //     rescale of O rows, and write each segment's partial O with coalesced stores.
 // QK : PV work is 576 : 512, so the two tensor pipes are nearly balanced and no FLOP or byte
 // is done twice (the second read of a page is an L2 hit).
+//
+// FP8 cache (e4m3 content codes, a fp32 scale per token, bf16 RoPE keys; the F8 instantiation):
+// each CTA dequantises the pages it needs, bf16(code * scale), into exactly the bf16 page tiles
+// the bf16 path loads, so everything after the page ring is shared.  The QK CTA's softmax warps
+// convert the next page before each page's softmax (2 page stages + 2 staging slots of raw
+// codes); four otherwise idle PV-CTA warps convert its half pages.
 //
 // Split-KV.  All (query row, page) units are spread evenly over the clusters (each cluster
 // works out its own contiguous range in its prologue, see schedule()); a range may cover parts
