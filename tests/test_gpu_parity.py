@@ -154,15 +154,16 @@ def test_append_fp8_codes_and_scales_are_bit_exact(oracle_mod):
         assert np.array_equal(scales[blk, slot].view(np.uint32), want_scales.view(np.uint32))
 
 
-def test_permuted_block_table_is_bitwise_identical():
-    wl = W.make_decode(33, [1000, 77, 640, 2048])
+@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+def test_permuted_block_table_is_bitwise_identical(kv):
+    wl = W.make_decode(33, [1000, 77, 640, 2048], kv_dtype=kv)
     a = GpuRun(wl)
     a.fill_cache()
     ga = a.step()
     rng = np.random.default_rng(5)
     perm = rng.permutation(wl.num_blocks + 3).astype(np.int32)
     bt = np.where(wl.block_table >= 0, perm[np.maximum(wl.block_table, 0)], -1).astype(np.int32)
-    wl2 = W.make_decode(33, [1000, 77, 640, 2048])
+    wl2 = W.make_decode(33, [1000, 77, 640, 2048], kv_dtype=kv)
     wl2.num_blocks = wl.num_blocks + 3
     b = GpuRun(wl2, block_table=bt)
     b.fill_cache()
@@ -171,8 +172,9 @@ def test_permuted_block_table_is_bitwise_identical():
         assert torch.equal(x, y)
 
 
-def test_repeated_decode_is_deterministic():
-    wl = W.make_decode(34, [4096, 100, 3000])
+@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+def test_repeated_decode_is_deterministic(kv):
+    wl = W.make_decode(34, [4096, 100, 3000], kv_dtype=kv)
     run = GpuRun(wl)
     run.fill_cache()
     g1 = run.step()
