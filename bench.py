@@ -59,6 +59,23 @@ def make_workload(name: str, batch: int | None = None):
     raise SystemExit(f"unknown config {name}")
 
 
+def max_over_ranks(values, world, device):
+    """Each rank's device times -> the max over all ranks (every rank gets it); the job's time
+    is the slowest replica's."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def job_tokens(tokens_per_rank: int, world: int) -> int:
+    """Query tokens one step of the whole job processes: every rank runs its own replica of the
+    batch (weak scaling)."""
+    return tokens_per_rank * world
+
+
 def algorithmic(wl):
     """Cache bytes and FLOPs of one mla_decode over the workload (per the method's definition:
     each query row reads its visible cache rows once; 2*(d_c+d_R) + 2*d_c FLOPs per head and
@@ -323,10 +340,7 @@ def run_mine(args):
     step_ms = sum(a.elapsed_time(b) for a, b in ev) / K
     dec_ms = sum(a.elapsed_time(b) for a, b in dev_ev) / K
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / K
-    t = torch.tensor([step_ms, dec_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    step_ms, dec_ms, e2e_ms = float(t[0]), float(t[1]), float(t[2])
+    step_ms, dec_ms, e2e_ms = max_over_ranks([step_ms, dec_ms, e2e_ms], world, dev)
     if N.mla_get_last_device_error() != 0:
         raise SystemExit("device error during the timed region")
     del g_step, g_dec, g_e2e
@@ -343,7 +357,7 @@ def run_mine(args):
     tfl = flops / dec_s / 1e12
     bound = "hbm" if cache_bytes / (hbm_peak * 1e9) >= flops / (tc_peak * 1e12) else "tensor"
     achieved, peak, unit = (gbs, hbm_peak, "GB/s") if bound == "hbm" else (tfl, tc_peak, "TFLOP/s")
-    tokens = T * world
+    tokens = job_tokens(T, world)
     if rank != 0:
         return
     line = {
