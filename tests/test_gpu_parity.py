@@ -172,6 +172,21 @@ def test_permuted_block_table_is_bitwise_identical(kv):
         assert torch.equal(x, y)
 
 
+@pytest.mark.parametrize("simt", [False, True], ids=["default", "simt"])
+def test_out_proj_bf16_output_is_the_rounded_f32_output(oracle_mod, simt):
+    """mla_out_proj with a bf16 output: the same fp32 accumulation, rounded once to bf16."""
+    wl = W.make_decode(38, [300, 65, 1], name="bf16_out")
+    run = GpuRun(wl, flags=3 if simt else 0)
+    run.fill_cache()
+    q_abs, o_lat, lse, o32 = run.step("f32")
+    o16 = run.layer.out_proj(o_lat, "bf16")
+    torch.cuda.synchronize()
+    assert o16.dtype == torch.bfloat16
+    assert torch.equal(o16, o32.to(torch.bfloat16))
+    rows, heads, ref = oracle_ref(wl, oracle_mod)
+    assert rel_l2(o16.float().cpu().numpy(), ref.o) <= BF16_REL
+
+
 @pytest.mark.parametrize("kv", ["bf16", "fp8"])
 def test_repeated_decode_is_deterministic(kv):
     wl = W.make_decode(34, [4096, 100, 3000], kv_dtype=kv)
