@@ -52,6 +52,8 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 
+#include <mutex>
+
 #include "mla_internal.cuh"
 #include "sm100.cuh"
 #include "tmap.cuh"
@@ -1315,12 +1317,16 @@ combine_tc_kernel(const int32_t *__restrict__ seg_range, const uint32_t *__restr
 
 // ---- host side ------------------------------------------------------------------------------
 int g_pairs[2][64] = {};
+std::mutex g_pairs_mu;
 
-// Co-resident clusters of the kernel on the current device (cached per device).
+// Co-resident clusters of the kernel on the current device (cached per device; the first call
+// on a device sets the kernel's shared-memory attribute and queries the occupancy, under a lock
+// so that concurrent first calls from several host threads do it once).
 template <bool F8>
 int tc_pairs() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    std::lock_guard<std::mutex> lk(g_pairs_mu);
     if (g_pairs[F8][dev]) return g_pairs[F8][dev];
     if (cudaFuncSetAttribute(decode_tc_kernel<F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay<F8>::smem) !=
         cudaSuccess)

@@ -1,5 +1,6 @@
 // C ABI entry points of libmla: host-side argument checks, then the launches.
 // The operations are documented in include/mla.h.
+#include <limits.h>
 #include <math.h>
 #include <mutex>
 #include <stdio.h>
@@ -131,6 +132,7 @@ mla_status_t mla_cache_append(const mla_dims_t *dims, int T, const void *c_kv, c
     if (T == 0) return MLA_OK;
     if (!c_kv || !k_r || !seq_idx || !pos || !block_table || !kv_pool) return MLA_ERR_INVALID_ARG;
     if (num_seqs == 0 || max_blocks_per_seq == 0 || num_blocks == 0) return MLA_ERR_INVALID_ARG;
+    if ((int64_t)max_blocks_per_seq * dims->page_size > INT_MAX) return MLA_ERR_INVALID_ARG;
     const bool fp8 = dims->kv_dtype == MLA_DTYPE_FP8_E4M3;
     if (fp8 != (kr_pool != nullptr) || fp8 != (kv_scale != nullptr)) return MLA_ERR_INVALID_ARG;
     return from_cuda(launch_append(*dims, T, c_kv, k_r, seq_idx, pos, block_table, num_seqs,
@@ -144,6 +146,7 @@ static bool use_tc(const mla_dims_t *d) {
 
 size_t mla_decode_workspace_size(const mla_dims_t *dims, int B, int s_q, int max_seq_len) {
     if (check_dims(dims) != MLA_OK || B < 0 || s_q < 1 || max_seq_len < 1) return 0;
+    if ((int64_t)B * s_q > INT_MAX) return 0;  // query rows are counted in int
     if (use_tc(dims)) return tc_workspace_bytes(*dims, B, s_q, max_seq_len);
     return simt_workspace_bytes(*dims, B, s_q, max_seq_len);
 }
@@ -158,6 +161,9 @@ mla_status_t mla_decode(const mla_dims_t *dims, int B, int s_q, const void *q_ab
     if (B < 0 || s_q < 1 || max_blocks_per_seq < 1 || num_blocks < 1 || max_seq_len < 1)
         return MLA_ERR_INVALID_ARG;
     if (B == 0) return MLA_OK;
+    // The kernels count query rows (B * s_q) and table positions (max_blocks * page) in int.
+    if ((int64_t)B * s_q > INT_MAX || (int64_t)max_blocks_per_seq * dims->page_size > INT_MAX)
+        return MLA_ERR_INVALID_ARG;
     if (max_seq_len > max_blocks_per_seq * dims->page_size || max_seq_len < s_q)
         return MLA_ERR_INVALID_ARG;
     if (!q_abs || !kv_pool || !block_table || !seq_lens || !workspace || !o_lat)

@@ -195,8 +195,10 @@ def varlen_decode(seed: int = 3, B: int = 64, lo: int = 1024, hi: int = 16384,
 def long_decode(seed: int = 4, B: int = 4, L: int = 131072) -> DecodeWorkload:
     """Long-context decode: rows [c_kv; k_R] = s_t z with z ~ N(0,1), s_t ~ LogNormal(0, 0.5)."""
     rng = np.random.default_rng(seed)
-    return _decode_workload("long_b%d_l%d" % (B, L), V3_DIMS, [L] * B, 1, "bf16", "bf16", rng,
-                            token_scale=lambda r, n: r.lognormal(0.0, 0.5, size=n))
+    wl = _decode_workload("long_b%d_l%d" % (B, L), V3_DIMS, [L] * B, 1, "bf16", "bf16", rng,
+                          token_scale=lambda r, n: r.lognormal(0.0, 0.5, size=n))
+    wl.extra["lognormal_norms"] = True
+    return wl
 
 
 def mtp_fp8_decode(seed: int = 5, B: int = 128, L: int = 8192, s_q: int = 2) -> DecodeWorkload:
@@ -215,8 +217,10 @@ def make_decode(seed: int, seq_lens, *, s_q: int = 1, kv_dtype: str = "bf16",
     tables, spare blocks, per-token norm spread)."""
     rng = np.random.default_rng(seed)
     ts = (lambda r, n: r.lognormal(0.0, 0.5, size=n)) if lognormal_tokens else None
-    return _decode_workload(name, dims, list(seq_lens), s_q, kv_dtype, act_dtype, rng,
-                            permute=permute, spare=spare, token_scale=ts)
+    wl = _decode_workload(name, dims, list(seq_lens), s_q, kv_dtype, act_dtype, rng,
+                          permute=permute, spare=spare, token_scale=ts)
+    wl.extra["lognormal_norms"] = bool(lognormal_tokens)
+    return wl
 
 
 CONFIGS = {

@@ -73,3 +73,36 @@ def decode(q_c, q_r, q_pos, c_kv, k_r, w_uk, w_uv, *, mode="absorbed", base=1e4)
         o_all.append(o_i)
         lse_all.append(lse_i)
     return o_all, lse_all
+
+
+def linear(w, x):
+    """y = W x for W given as rows [out][in] (the nn.Linear weight convention), by loops."""
+    return [sum(w[o][k] * x[k] for k in range(len(x))) for o in range(len(w))]
+
+
+def toy_projections(h, W):
+    """Projections of the simplified layer for one sequence h [T][d], by loops, written from
+    the notation of sections 구조 and 분리 RoPE rather than from any reshape:
+        c^KV_t = W^DKV h_t,   k^R_t = W^KR h_t   (the shared RoPE key comes from h_t),
+        c^Q_t  = W^DQ h_t,
+        q^C_{t,i} = W^UQ_i c^Q_t,   q^R_{t,i} = W^QR_i c^Q_t,
+    where W^UQ_i (W^QR_i) is the i-th block of d_h (d_R) consecutive rows of W^UQ (W^QR): head i
+    owns output features i*d_h .. i*d_h + d_h - 1 (section 행렬 흡수's per-head W_i).
+    Returns (c_kv [T][d_c], k_r [T][d_R], q_c [T][n_h][d_h], q_r [T][n_h][d_R]); keys and
+    queries before RoPE."""
+    n_h, d_h, d_r = W["n_h"], W["d_h"], W["d_r"]
+    c_kv, k_r, q_c, q_r = [], [], [], []
+    for x in h:
+        c_kv.append(linear(W["w_dkv"], x))
+        k_r.append(linear(W["w_kr"], x))
+        cq = linear(W["w_dq"], x)
+        q_c.append([linear(W["w_uq"][i * d_h:(i + 1) * d_h], cq) for i in range(n_h)])
+        q_r.append([linear(W["w_qr"][i * d_r:(i + 1) * d_r], cq) for i in range(n_h)])
+    return c_kv, k_r, q_c, q_r
+
+
+def output_projection(o_heads, w_o):
+    """u_t = W^O [o_{t,1}; ...; o_{t,n_h}] for one token: the heads' outputs concatenated in
+    head order (section 분리 RoPE, output equation), then W^O [d][n_h*d_h]."""
+    cat = [v for head in o_heads for v in head]
+    return linear(w_o, cat)

@@ -18,7 +18,12 @@ def max_abs(x, ref) -> float:
     return float(np.max(np.abs(np.asarray(x, dtype=np.float64) - np.asarray(ref, dtype=np.float64))))
 
 
-# Tolerances (see test_gpu_parity.py's module docstring for their reading).
+# Tolerances of the bf16 path: relative L2 <= 4e-3 and max |err| <= 2e-2 on o_lat and o, and
+# |err(lse)| <= 1e-2.  Workloads whose per-token norms are log-normal (the long-context recipe)
+# use max |err| <= 2e-2 * max(1, max |ref|) and |err(lse)| <= 1e-2 * max(1, |lse|) instead:
+# tests/test_tolerance_reading.py shows that exact arithmetic on the bf16 operands the C ABI
+# defines already exceeds the flat bounds there, and stays far inside them on N(0,1) latents.
+# FP8 content cache: relative L2 <= 3e-2 against the oracle on its own dequantised cache.
 BF16_REL, BF16_ABS, FP8_REL, LSE_ABS = 4e-3, 2e-2, 3e-2, 1e-2
 
 
@@ -29,19 +34,27 @@ def scaled_max_abs(x, ref):
     return float(np.abs(x - ref).max() / max(1.0, float(np.abs(ref).max())))
 
 
-def check_step(got, ref, rows, heads, rel_tol, abs_tol):
-    """Compare one step's (o_lat, lse, o) on the given rows and heads with the oracle's."""
+def check_step(got, ref, rows, heads, rel_tol, abs_tol, *, lognormal=False):
+    """Compare one step's (o_lat, lse, o) on the given rows and heads with the oracle's.
+
+    ``lognormal``: the workload's per-token norms are log-normal; the max-abs and lse bounds
+    scale with the output (see the tolerance note above).  Both the plain and the scaled
+    errors are always reported in the assertion message."""
     q_abs, o_lat, lse, o = got
     o_lat = o_lat.cpu().numpy()[rows][:, heads]
     o = o.float().cpu().numpy()[rows][:, heads]
     lse = lse.cpu().numpy()[rows][:, heads]
+    dl = np.abs(lse.astype(np.float64) - ref.lse)
     e = dict(o_lat_rel=rel_l2(o_lat, ref.o_lat), o_rel=rel_l2(o, ref.o),
-             o_lat_abs=scaled_max_abs(o_lat, ref.o_lat), o_abs=scaled_max_abs(o, ref.o),
-             lse_abs=float(np.max(np.abs(lse - ref.lse) / np.maximum(1.0, np.abs(ref.lse)))))
+             o_lat_abs=max_abs(o_lat, ref.o_lat), o_abs=max_abs(o, ref.o),
+             o_lat_scaled=scaled_max_abs(o_lat, ref.o_lat), o_scaled=scaled_max_abs(o, ref.o),
+             lse_abs=float(dl.max()), lse_scaled=float(np.max(dl / np.maximum(1.0, np.abs(ref.lse)))),
+             bounds="scaled (log-normal norms)" if lognormal else "flat")
     assert e["o_lat_rel"] <= rel_tol and e["o_rel"] <= rel_tol, e
+    k = "_scaled" if lognormal else "_abs"
     if abs_tol is not None:
-        assert e["o_lat_abs"] <= abs_tol and e["o_abs"] <= abs_tol, e
-    assert e["lse_abs"] <= LSE_ABS, e
+        assert e["o_lat" + k] <= abs_tol and e["o" + k] <= abs_tol, e
+    assert e["lse" + k] <= LSE_ABS, e
     return e
 
 

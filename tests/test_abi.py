@@ -69,6 +69,14 @@ def test_host_argument_checks(N):
     assert L.mla_decode(*args) == N.MLA_ERR_WORKSPACE_TOO_SMALL
     args = [dp, 2, 1, 16, 16, None, None, 16, 4, 8, 16, 256, 8, 1 << 30, 16, 16, None]
     assert L.mla_decode(*args) == N.MLA_ERR_INVALID_ARG
+    # query rows (B * s_q) and table positions (max_blocks * page) must fit in int
+    sp = ctypes.byref(simt)
+    args = [sp, 1 << 20, 1 << 12, 16, 16, None, None, 16, 4, 8, 16, 256, 256, 1 << 40, 16, 16, None]
+    assert L.mla_decode(*args) == N.MLA_ERR_INVALID_ARG
+    args = [sp, 2, 1, 16, 16, None, None, 16, 1 << 26, 8, 16, 256, 256, 1 << 40, 16, 16, None]
+    assert L.mla_decode(*args) == N.MLA_ERR_INVALID_ARG
+    assert N.mla_decode_workspace_size(simt, 1 << 20, 1 << 12, 4096) == 0
+    assert L.mla_cache_append(dp, 1, 8, 8, 8, 8, 8, 1, 1 << 26, 1, 8, None, None, None) == N.MLA_ERR_INVALID_ARG
 
 
 def test_workspace_size_is_positive_and_monotone(N):

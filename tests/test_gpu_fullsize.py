@@ -45,4 +45,5 @@ def test_full_size_sampled_rows(oracle_mod, cfg):
     heads = np.sort(rng.choice(wl.dims.n_h, n_head, replace=False))
     rows, heads, ref = oracle_ref(wl, oracle_mod, seqs, heads)
     fp8 = wl.kv_dtype == "fp8"
-    check_step(got, ref, rows, heads, FP8_REL if fp8 else BF16_REL, None if fp8 else BF16_ABS)
+    check_step(got, ref, rows, heads, FP8_REL if fp8 else BF16_REL, None if fp8 else BF16_ABS,
+               lognormal=wl.extra.get("lognormal_norms", False))

@@ -1,14 +1,12 @@
 """GPU parity of the CUDA path (through the C ABI) against the fp64 CPU oracle.
 
-Tolerances.  bf16 path: relative L2 <= 4e-3 and max |err| <= 2e-2 * max(1, max |ref|) on
-o_lat and o (the normalised infinity-norm error): for O(1) outputs (N(0,1) latents) this is
-the plain 2e-2 bound; outputs of the log-normal-norm workload reach |o_lat| ~ 20, where
-rounding the absorbed query to bf16 alone (an fp64 emulation) already moves single elements
-by ~0.1, so the bound scales with the output's magnitude.  FP8
-content cache: relative L2 <= 3e-2 against the oracle run on its own dequantised cache
-(the same codes, checked bit-exact below); lse within 1e-2 * max(1, |lse|) (its bf16 error
-grows with the score magnitude: 0.018 on the log-normal workload's lse of 9..19).  The fp32 toy layer
-accumulates in fp32 over at most 256 tokens x 160 dims: relative L2 <= 1e-5.
+Tolerances.  bf16 path: relative L2 <= 4e-3, max |err| <= 2e-2 on o_lat and o, |err(lse)|
+<= 1e-2.  Cases whose per-token norms are log-normal use max |err| <= 2e-2 * max(1, max |ref|)
+and |err(lse)| <= 1e-2 * max(1, |lse|): exact arithmetic on the bf16 operands of the C ABI
+already moves single elements of o_lat by ~0.1 and lse by ~0.02 there
+(tests/test_tolerance_reading.py).  FP8 content cache: relative L2 <= 3e-2 against the oracle
+run on its own dequantised cache (the same codes, checked bit-exact below).  The fp32 toy
+layer accumulates in fp32 over at most 256 tokens x 160 dims: relative L2 <= 1e-5.
 """
 import numpy as np
 import pytest
@@ -32,7 +30,8 @@ def _cuda():
 
 
 def _check(wl, got, ref, rows, heads, rel_tol, abs_tol):
-    return check_step(got, ref, rows, heads, rel_tol, abs_tol)
+    return check_step(got, ref, rows, heads, rel_tol, abs_tol,
+                      lognormal=wl.extra.get("lognormal_norms", False))
 
 
 # ---------------------------------------------------------------------------------------------

@@ -216,6 +216,54 @@ def test_brute_force_loops_match_oracle(oracle_mod, mode):
 # FP8 e4m3 codec against torch's float8_e4m3fn
 # ---------------------------------------------------------------------------------------------
 
+def _tiny_toy_weights(seed):
+    """Tiny simplified-layer weights with d_cq == d, so that taking k^R from c^Q instead of h
+    (or any other mix-up of the two inputs) still runs and shows up only in the values."""
+    rng = np.random.default_rng(seed)
+    d, n_h, d_h, d_c, d_cq, d_r = 5, 3, 2, 4, 5, 4
+    w = lambda o, i: rng.standard_normal((o, i)) / np.sqrt(i)
+    return dict(n_h=n_h, d_h=d_h, d_r=d_r, d_c=d_c, d=d, d_cq=d_cq,
+                w_dq=w(d_cq, d), w_uq=w(n_h * d_h, d_cq), w_qr=w(n_h * d_r, d_cq), w_dkv=w(d_c, d),
+                w_kr=w(d_r, d), w_uk=w(n_h * d_h, d_c), w_uv=w(n_h * d_h, d_c), w_o=w(d, n_h * d_h))
+
+
+def test_toy_projections_match_per_head_loops(oracle_mod):
+    """The oracle's up projections split the n_h*d_h features head by head (head i owns rows
+    i*d_h ..), and the RoPE key is projected from h, as the loops written from the sections'
+    notation do.  A feature split in the other order, or k^R taken from c^Q, fails here."""
+    Wt = _tiny_toy_weights(11)
+    h = np.random.default_rng(12).standard_normal((1, 4, Wt["d"]))
+    c_kv, k_r, q_c, q_r = oracle_mod.toy_projections(h, Wt)
+    bc, bk, bq, br = brute.toy_projections(h[0].tolist(), {k: (v.tolist() if hasattr(v, "tolist") else v)
+                                                          for k, v in Wt.items()})
+    for got, want in ((c_kv[0], bc), (k_r[0], bk), (q_c[0], bq), (q_r[0], br)):
+        assert np.max(np.abs(np.asarray(got) - np.asarray(want))) <= 1e-13
+    # the planted mistakes really differ
+    n_h, d_h, d_r = Wt["n_h"], Wt["d_h"], Wt["d_r"]
+    cq = h[0] @ Wt["w_dq"].T
+    wrong_split = (cq @ Wt["w_uq"].T).reshape(4, d_h, n_h).transpose(0, 2, 1)
+    assert np.max(np.abs(wrong_split - np.asarray(bq))) > 1e-2
+    assert np.max(np.abs(cq @ Wt["w_kr"].T - np.asarray(bk))) > 1e-2
+
+
+def test_toy_layer_output_projection_matches_loops(oracle_mod):
+    """u = W^O [o_1; ...; o_{n_h}] over the whole simplified layer (prefill form, every token
+    querying): the oracle against the loops end to end (projections, decode, W^O)."""
+    Wt = _tiny_toy_weights(13)
+    T = 5
+    h = np.random.default_rng(14).standard_normal((1, T, Wt["d"]))
+    res = oracle_mod.toy_layer(h, Wt, mode="absorbed", last_only=False)
+    L = {k: (v.tolist() if hasattr(v, "tolist") else v) for k, v in Wt.items()}
+    bc, bk, bq, br = brute.toy_projections(h[0].tolist(), L)
+    o, _ = brute.decode(bq, br, list(range(T)), bc, bk, L["w_uk"], L["w_uv"], mode="naive")
+    u = [brute.output_projection(o[t], L["w_o"]) for t in range(T)]
+    assert np.max(np.abs(res.u[0] - np.asarray(u))) <= 1e-12
+    # a head-interleaved concatenation (feature d of every head, then d + 1, ...) differs
+    o_arr = np.asarray(o)
+    wrong = o_arr.transpose(0, 2, 1).reshape(T, -1) @ Wt["w_o"].T
+    assert np.max(np.abs(wrong - np.asarray(u))) > 1e-2
+
+
 def test_e4m3_table_matches_library(oracle_mod):
     lib_vals = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
     mine = np.array([oracle_mod.e4m3_value(c) for c in range(256)])

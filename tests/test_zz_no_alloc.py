@@ -3,20 +3,21 @@ against mla_decode with a caller workspace, through the C ABI.
 
 The file name sorts last so that the test also runs after every other test in one session;
 it passes alone in a fresh process as well (the first call on the device does the scratch
-set-up).  Tolerance: the bf16 parity bound of the other GPU tests (relative L2 <= 4e-3);
-both calls run the same kernels, so in practice the results agree bit for bit.
+set-up).  Both entry points run the same kernels on the same inputs, so their results must
+agree bit for bit.  The scratch array keeps the previous call's contents; the test first
+fills it with a call on a larger, different batch, so that a kernel that read a partial slot
+or a slot range it did not write in the current call would show up as a difference.  The
+target batch has fewer pages than the kernel has clusters, so some clusters sit inside a
+row's slot range with no pages of it and must mark their slot empty in every call.
 """
 import numpy as np
 import pytest
 import torch
 
 from mla_latent_kv_mqa_b200 import workloads as W
-from tests.harness import GpuRun, rel_l2
+from tests.harness import GpuRun
 
 pytestmark = pytest.mark.gpu
-
-REL = 4e-3
-
 
 @pytest.fixture(scope="module", autouse=True)
 def _cuda():
@@ -43,6 +44,15 @@ def _fixed_scratch_decode(run, q_abs):
 @pytest.mark.parametrize("flags", [0, 1], ids=["tensor_core", "simt"])
 def test_fixed_scratch_matches_workspace_decode_twice(flags):
     from mla_latent_kv_mqa_b200 import native as N
+    # a different, larger batch first: every slot it writes holds stale values afterwards
+    other = W.make_decode(43, [int(x) for x in np.random.default_rng(43).integers(1, 2500, 40)],
+                          permute=True, spare=3)
+    orun = GpuRun(other, flags=flags)
+    orun.fill_cache()
+    oq = orun.layer.absorb(orun.q_c, orun.q_r, orun.q_pos)
+    o_other, _ = _fixed_scratch_decode(orun, oq)
+    assert torch.isfinite(o_other).all()
+
     wl = W.make_decode(41, [700, 33, 1000, 64 * 5, 1], permute=True, spare=8)
     run = GpuRun(wl, flags=flags)
     run.fill_cache()
@@ -50,13 +60,11 @@ def test_fixed_scratch_matches_workspace_decode_twice(flags):
     ref_o, ref_lse = run.layer.decode(run.cache, q_abs, run.block_table, run.seq_lens, wl.s_q,
                                       run.max_seq_len)
     torch.cuda.synchronize()
-    ref_o, ref_lse = ref_o.cpu().numpy(), ref_lse.cpu().numpy()
+    assert torch.isfinite(ref_o).all() and torch.isfinite(ref_lse).all()
     for _ in range(2):  # two calls in a row share the scratch array
         o, lse = _fixed_scratch_decode(run, q_abs)
-        o, lse = o.cpu().numpy(), lse.cpu().numpy()
-        assert np.isfinite(o).all() and np.isfinite(lse).all()
-        assert rel_l2(o, ref_o) <= REL
-        assert rel_l2(lse, ref_lse) <= REL
+        assert torch.equal(o, ref_o)
+        assert torch.equal(lse, ref_lse)
     assert N.mla_get_last_device_error() == N.MLA_OK
 
 
