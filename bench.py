@@ -32,6 +32,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "absorbed-MLA decode tokens/s; latent-cache GB/s & TFLOP/s vs B200 roofline"
 WORKLOADS = {
+    "toy": "Toy MLA layer (page-5 dims): d=1024, n_h=8, d_h=64, d_c=128, d_cq=256, d_R=32, batch 1, "
+           "context 256, s_q=1, fp32",
     "v3": "DeepSeek-V3-shaped single layer decode: n_h=128, d_h=128, d_c=512, d_R=64, bf16 latent "
           "cache, batch 16, uniform context 4096, s_q=1, page 64",
     "varlen": "V3 dims, batch 64, context U[1024,16384], permuted block table, bf16",
@@ -48,6 +50,10 @@ DECODE_TRAFFIC = {"v3": 78050048 + 2524160}
 
 def make_workload(name: str, batch: int | None = None):
     from mla_latent_kv_mqa_b200 import workloads as W
+    if name == "toy":
+        # The toy layer's decode inputs: activations N(0, 1) (what W^DKV h, W^UQ W^DQ h, ... give
+        # for h ~ N(0, 1) and nn.Linear weights ~ N(0, 1/fan_in)), W^UK, W^UV ~ N(0, 1/d_c), fp32.
+        return W.make_decode(1, [256], dims=W.TOY_DIMS, act_dtype="f32", kv_dtype="f32", name="toy")
     if name == "v3":
         return W.v3_decode(B=batch or 16)
     if name == "varlen":
@@ -158,12 +164,16 @@ class ClockSampler:
                 "window": "the last 0.5 s of the sustained warm-up load and the timed region"}
 
 
-def cpu_baseline(wl, budget_s: float = 12.0):
-    """The fp64 oracle (absorbed mode), as it stands, on a bounded sample of the workload:
-    whole sequences (all heads, all visible tokens) until ``budget_s`` is spent."""
+def cpu_baseline(wl, budget_s: float = 8.0, single_budget_s: float = 3.0):
+    """The fp64 oracle (absorbed mode), as it stands, on a bounded sample of the workload: whole
+    sequences (all heads, all visible tokens) until ``budget_s`` is spent, with the oracle's
+    default host threads; then single-threaded on the first sequence, on as many heads as fit
+    in about ``single_budget_s`` (scaled to all heads)."""
+    import numpy as _np
     from oracle import oracle as orc
     from tests.harness import oracle_ref
     orc.build()
+    threads = orc.num_threads()
     t0 = time.perf_counter()
     n_seq = 0
     for b in range(wl.B):
@@ -172,8 +182,35 @@ def cpu_baseline(wl, budget_s: float = 12.0):
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
-    return {"value": n_seq * wl.s_q / dt, "unit": "tokens/s", "cores": orc.num_threads(), "kind": "oracle",
-            "sample": f"{n_seq} of {wl.B} sequences, all {wl.dims.n_h} heads, fp64 absorbed mode, {dt:.1f} s"}
+    # single thread, on sequence 0's prepared inputs (the cache rows as the oracle reads them,
+    # FP8 ones dequantised), so that only the decode itself is timed: one head first, then as
+    # many heads as fit in the budget
+    from tests.harness import oracle_cache_rows
+    d = wl.dims
+    cs, ks = oracle_cache_rows(wl, orc, [0])
+    rows = _np.arange(wl.s_q)
+
+    def one(nh):
+        hs = _np.arange(nh)
+        wsel = (hs[:, None] * d.d_h + _np.arange(d.d_h)[None, :]).reshape(-1)
+        t = time.perf_counter()
+        orc.decode_absorbed(wl.q_c[rows][:, hs], wl.q_r[rows][:, hs], wl.q_pos[rows], cs, ks,
+                            wl.w_uk[wsel], wl.w_uv[wsel], s_q=wl.s_q, rope_base=d.rope_base)
+        return time.perf_counter() - t
+
+    orc.set_num_threads(1)
+    try:
+        t_one = one(1)
+        nh = int(max(1, min(d.n_h, single_budget_s / max(t_one, 1e-6))))
+        st = one(nh)
+    finally:
+        orc.set_num_threads(threads)
+    st_tok = wl.s_q / (st * wl.dims.n_h / nh)  # query tokens/s with all heads, one thread
+    return {"value": n_seq * wl.s_q / dt, "unit": "tokens/s", "cores": threads, "nproc": os.cpu_count(),
+            "threads": threads, "kind": "oracle",
+            "sample": f"{n_seq} of {wl.B} sequences, all {wl.dims.n_h} heads, fp64 absorbed mode, {dt:.1f} s",
+            "single_thread": {"value": st_tok, "unit": "tokens/s",
+                              "sample": f"sequence 0, {nh} of {wl.dims.n_h} heads, {st:.1f} s, scaled to all heads"}}
 
 
 def run_reference(args):
@@ -214,31 +251,24 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def run_mine(args):
+def peaks_of():
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return peaks["hbm_gbs"], peaks["bf16_tflops"], "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, "fallback"
+
+
+def measure(name, K, warmup, world, dev, clock_warmup_s, with_clock=True):
+    """Time one workload: K steps of the whole path (CUDA graph, L2 flushed before each step),
+    K decode-only replays, K end-to-end steps from pinned host buffers.  Returns a dict (device
+    times already reduced to the max over ranks) and the workload."""
     import torch
     import torch.distributed as dist
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        from datetime import timedelta
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
-    dev = torch.device("cuda", torch.cuda.current_device())
-
-    from mla_latent_kv_mqa_b200 import build
-    if rank == 0:
-        build.build()
-    if world > 1:
-        dist.barrier()
-    from mla_latent_kv_mqa_b200 import layer as Lyr
     from mla_latent_kv_mqa_b200 import native as N
     from tests.harness import GpuRun
 
-    wl = make_workload(args.config)
+    wl = make_workload(name)
     run = GpuRun(wl, dev=dev)
     run.fill_cache()
     L = run.layer
@@ -253,7 +283,7 @@ def run_mine(args):
     o_lat = torch.empty((T, wl.dims.n_h, wl.dims.d_c), dtype=torch.float32, device=dev)
     lse = torch.empty((T, wl.dims.n_h), dtype=torch.float32, device=dev)
     o = torch.empty((T, wl.dims.n_h, wl.dims.d_h), dtype=torch.float32, device=dev)
-    ws = L.workspace(B, s_q, run.max_seq_len)
+    L.workspace(B, s_q, run.max_seq_len)
     decode_launches = 2  # split-KV main kernel + log-sum-exp combine
     launches_per_step = 1 + 1 + decode_launches + 1
 
@@ -292,13 +322,13 @@ def run_mine(args):
         h_out.copy_(o, non_blocking=True)
 
     with torch.cuda.stream(stream):
-        for _ in range(max(args.warmup, 3)):  # eager warm-up (also sets up kernel attributes)
+        for _ in range(max(warmup, 3)):  # eager warm-up (also sets up kernel attributes)
             flush.fill_(1)
             step()
             e2e_step()
         stream.synchronize()
         if N.mla_get_last_device_error() != 0:
-            raise SystemExit("device error during warm-up")
+            raise SystemExit(f"device error during warm-up ({name})")
         g_step, g_dec, g_e2e = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_step, stream=stream):
             step()
@@ -306,20 +336,19 @@ def run_mine(args):
             decode_only()
         with torch.cuda.graph(g_e2e, stream=stream):
             e2e_step()
-        for _ in range(max(args.warmup, 3)):  # graph warm-up
+        for _ in range(max(warmup, 3)):  # graph warm-up
             flush.fill_(2)
             g_step.replay()
             g_dec.replay()
             g_e2e.replay()
         stream.synchronize()
-        K = args.steps
         mk = lambda: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
         ev, dev_ev, e2e_ev = mk(), mk(), mk()
         bus = torch.cuda.get_device_properties(dev).pci_bus_id
-        with ClockSampler(bus) as clk:
+        with ClockSampler(bus if with_clock else -1) as clk:
             # let the SM clock ramp up under sustained load before timing (idle boards sit far below
             # boost); the clock samples of its last half second count with the timed region's
-            t_end = time.time() + max(args.clock_warmup_s, 0.8)
+            t_end = time.time() + max(clock_warmup_s, 0.8)
             while time.time() < t_end:
                 for _ in range(20):
                     g_step.replay()
@@ -355,49 +384,113 @@ def run_mine(args):
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / K
     step_ms, dec_ms, e2e_ms = max_over_ranks([step_ms, dec_ms, e2e_ms], world, dev)
     if N.mla_get_last_device_error() != 0:
-        raise SystemExit("device error during the timed region")
+        raise SystemExit(f"device error during the timed region ({name})")
     del g_step, g_dec, g_e2e
+    res = dict(step_ms=step_ms, dec_ms=dec_ms, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
+               launches=(launches_per_step + decode_launches) * K, clocks=clk.summary() if with_clock else None)
+    del run, flush, h_pack, d_pack, h_out
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res, wl
 
+
+def roofline_of(wl, dec_ms):
+    hbm_peak, tc_peak, src = peaks_of()
     cache_bytes, flops = algorithmic(wl)
-    peaks = {}
-    try:
-        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
-        hbm_peak, tc_peak, src = peaks["hbm_gbs"], peaks["bf16_tflops"], "measured"
-    except (OSError, KeyError, ValueError):
-        hbm_peak, tc_peak, src = 6650.0, 1590.0, "fallback"
     dec_s = dec_ms * 1e-3
     gbs = cache_bytes / dec_s / 1e9
     tfl = flops / dec_s / 1e12
+    # the fp32 toy layer runs on CUDA cores: its binding peak is not the bf16 tensor one
     bound = "hbm" if cache_bytes / (hbm_peak * 1e9) >= flops / (tc_peak * 1e12) else "tensor"
     achieved, peak, unit = (gbs, hbm_peak, "GB/s") if bound == "hbm" else (tfl, tc_peak, "TFLOP/s")
-    tokens = job_tokens(T, world)
-    if rank != 0:
-        return
-    line = {
-        "metric": METRIC, "value": tokens / (step_ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
-        "steps": K, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.kv_dtype == "bf16" else wl.kv_dtype,
-        "data": "synthetic",
-        "config": {"workload": WORKLOADS[args.config], "batch_per_gpu": B, "s_q": s_q,
-                   "context": int(wl.seq_lens.max()), "parallelism": f"replicas x{world}",
-                   "l2": "flushed before every timed step (512 MiB write outside the events)",
-                   "launch": "each step is one CUDA-graph replay of the four calls"},
-        "decode": {"kernel": "mla_decode (tcgen05 split-KV main with in-kernel schedule + LSE combine)",
-                   "ms": dec_ms, "tokens_per_s": tokens / dec_s, "cache_gbs": gbs, "tflops": tfl,
-                   "frac_hbm": gbs / hbm_peak, "frac_bf16": tfl / tc_peak,
-                   "cache_bytes": cache_bytes, "flops": flops},
-        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak, "traffic": DECODE_TRAFFIC.get(args.config), "peak_source": src,
-                     "kernel": "mla_decode", "algorithmic_per_launch": cache_bytes if bound == "hbm" else flops},
-        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "how": "CUDA graph of one pinned H2D copy of the packed inputs + the four calls + D2H of o; host reads o each step"},
-        "gpu_launches": (launches_per_step + decode_launches) * K,
-        "clocks": clk.summary(),
-    }
-    if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl)
-    print(json.dumps(line), flush=True)
+    return dict(cache_bytes=cache_bytes, flops=flops, gbs=gbs, tfl=tfl, bound=bound, achieved=achieved,
+                peak=peak, unit=unit, frac=achieved / peak, src=src, hbm_peak=hbm_peak, tc_peak=tc_peak)
+
+
+def run_mine(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    from mla_latent_kv_mqa_b200 import build
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+
+    K = args.steps
+    r, wl = measure(args.config, K, args.warmup, world, dev, args.clock_warmup_s)
+    rf = roofline_of(wl, r["dec_ms"])
+    tokens = job_tokens(wl.T, world)
+    line = None
+    if rank == 0:
+        dtype = {"bf16": "bf16", "f32": "f32"}.get(wl.kv_dtype, wl.kv_dtype)
+        line = {
+            "metric": METRIC, "value": tokens / (r["step_ms"] * 1e-3), "unit": "tokens/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": r["step_ms"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+            "config": {"workload": WORKLOADS[args.config], "batch_per_gpu": wl.B, "s_q": wl.s_q,
+                       "context": int(wl.seq_lens.max()), "parallelism": f"replicas x{world}",
+                       "l2": "flushed before every timed step (512 MiB write outside the events)",
+                       "launch": "each step is one CUDA-graph replay of the four calls"},
+            "decode": {"kernel": "mla_decode (tcgen05 split-KV main with in-kernel schedule + LSE combine)",
+                       "ms": r["dec_ms"], "tokens_per_s": tokens / (r["dec_ms"] * 1e-3), "cache_gbs": rf["gbs"],
+                       "tflops": rf["tfl"], "frac_hbm": rf["gbs"] / rf["hbm_peak"],
+                       "frac_bf16": rf["tfl"] / rf["tc_peak"], "cache_bytes": rf["cache_bytes"], "flops": rf["flops"]},
+            "roofline": {"bound": rf["bound"], "achieved": rf["achieved"], "peak": rf["peak"], "unit": rf["unit"],
+                         "frac": rf["frac"], "traffic": DECODE_TRAFFIC.get(args.config), "peak_source": rf["src"],
+                         "kernel": "mla_decode",
+                         "algorithmic_per_launch": rf["cache_bytes"] if rf["bound"] == "hbm" else rf["flops"]},
+            "e2e": {"value": tokens / (r["e2e_ms"] * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"],
+                    "d2h_bytes_per_step": r["d2h"], "ms_per_step": r["e2e_ms"],
+                    "how": "CUDA graph of one pinned H2D copy of the packed inputs + the four calls + D2H of o; host reads o each step"},
+            "gpu_launches": r["launches"],
+            "clocks": r["clocks"],
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl)
+    del wl
+    # The other workloads, each measured the same way with fewer steps (one GPU only: under
+    # torchrun every rank would hold every workload and the scaling run would take minutes).
+    if world == 1 and not args.only:
+        configs = {}
+        k2 = max(5, K // 4)
+        for name in WORKLOADS:
+            if name == args.config:
+                continue
+            r2, wl2 = measure(name, k2, args.warmup, world, dev, 0.8)
+            rf2 = roofline_of(wl2, r2["dec_ms"])
+            t2 = job_tokens(wl2.T, world)
+            c = {"workload": WORKLOADS[name], "steps": k2, "step_ms": r2["step_ms"],
+                 "tokens_per_s": t2 / (r2["step_ms"] * 1e-3),
+                 "decode_ms": r2["dec_ms"], "decode_tokens_per_s": t2 / (r2["dec_ms"] * 1e-3),
+                 "cache_gbs": rf2["gbs"], "tflops": rf2["tfl"], "frac_hbm": rf2["gbs"] / rf2["hbm_peak"],
+                 "frac_bf16": rf2["tfl"] / rf2["tc_peak"],
+                 "roofline": {"bound": rf2["bound"], "frac": rf2["frac"], "peak": rf2["peak"], "unit": rf2["unit"],
+                              "traffic": DECODE_TRAFFIC.get(name), "peak_source": rf2["src"]},
+                 "e2e": {"value": t2 / (r2["e2e_ms"] * 1e-3), "unit": "tokens/s", "ms_per_step": r2["e2e_ms"],
+                         "h2d_bytes_per_step": r2["h2d"], "d2h_bytes_per_step": r2["d2h"]},
+                 "gpu_launches": r2["launches"], "clocks": r2["clocks"]}
+            if name == "toy":
+                c["roofline"]["note"] = ("fp32 layer on the CUDA-core decode kernel: launch-bound at 256 "
+                                         "tokens; the fraction is reported against the bf16 peaks as is")
+            if not args.no_cpu_baseline:
+                c["cpu_baseline"] = cpu_baseline(wl2)
+            configs[name] = c
+            del wl2
+        line["configs"] = configs
+    if rank == 0:
+        print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
 
@@ -426,6 +519,7 @@ def main():
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
     ap.add_argument("--config", default="v3", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", action="store_true", help="time only --config (no per-workload block)")
     ap.add_argument("--plain-steps", type=int, default=0, help="run N untimed eager steps and exit (profiling)")
     ap.add_argument("--batch", type=int, default=None, help="with --plain-steps: batch of the v3 or mtp_fp8 workload")
     args = ap.parse_args()

@@ -85,6 +85,14 @@ typedef enum {
 #define MLA_FLAG_SIMT_DECODE 1u /* run mla_decode on the CUDA-core kernel even where the
                                    tensor-core kernel applies (cross-checks) */
 #define MLA_FLAG_SIMT_PROJ 2u   /* same for mla_absorb_q and mla_out_proj */
+#define MLA_FLAG_TEST_GIVE_UP 4u /* test of the failure path of the tensor-core decode: in
+                                    every cluster with two or more pages, after the copies of
+                                    the first page have started, one bounded wait (20 us) on a
+                                    barrier that nothing completes gives up.  The cluster then
+                                    does what any timed-out wait does: it flags both of its CTAs,
+                                    records MLA_ERR_DEVICE_TIMEOUT in the device error word,
+                                    waits (2 s bound) for the copies and MMAs it has started, and
+                                    exits.  The call's outputs are invalid; nothing faults. */
 
 typedef struct {
     int n_h;            /* heads */

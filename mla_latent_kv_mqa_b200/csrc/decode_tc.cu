@@ -130,6 +130,7 @@ struct __align__(8) Ctrl {
     uint64_t vstg_full[2], vstg_empty[2];   // FP8: raw half-page codes landed / converted
     uint64_t corr_done, o_free;
     uint64_t mma_idle[2];       // drains: one per MMA-issuing thread
+    uint64_t never_done;        // test of the failure path: a barrier that nothing completes
     uint32_t tmem_base;
     uint32_t abort;
     uint32_t never;             // stays 0: the abort word of drain waits, which must not give up early
@@ -164,6 +165,7 @@ struct Params {
     float *m_part, *l_part;
     float scale_log2;
     unsigned *err;
+    int test_give_up;         // MLA_FLAG_TEST_GIVE_UP: the QK producer gives up before its second page
     const uint8_t *codes;     // FP8: content codes [num_blocks][64][512]
     const float *kv_scale;    // FP8: per-token scales [num_blocks][64]
 };
@@ -379,9 +381,50 @@ __device__ __forceinline__ long long block_scan(int x, Ctrl *ctrl, long long &to
     __syncthreads();
     return before + x;
 }
+// The cluster holding unit u (the inverse of unit_start).
+__device__ __forceinline__ int pair_of_unit(long long u, long long U, int pairs) {
+    int c = (int)(u * pairs / U);
+    while (c + 1 < pairs && unit_start(c + 1, U, pairs) <= u) ++c;
+    while (c > 0 && unit_start(c, U, pairs) > u) --c;
+    return c;
+}
+// Row r has n > 0 units starting at unit u0: record this cluster's work if it starts inside the
+// row, mark this cluster's slot empty if the row's slot range covers it but it got no units,
+// and (cluster 0) write the row's slot range.
+__device__ __forceinline__ void schedule_row(const Params &P, int pair, uint32_t rank, Ctrl *ctrl, int r, int n,
+                                             long long u0, long long U, long long s0, long long s1) {
+    if (n > 0 && u0 <= s0 && s0 < u0 + n) {  // the row holding unit s0
+        if (s1 > s0) {
+            ctrl->w_r0 = r;
+            ctrl->w_pg0 = (int)(s0 - u0);
+        } else if (rank == 0) {
+            for (int h = 0; h < NH; ++h) P.m_part[((size_t)pair + r) * NH + h] = -INFINITY;
+        }
+    }
+    if (pair == 0 && rank == 0 && r < P.rows) {
+        P.seg_range[2 * r] = n > 0 ? pair_of_unit(u0, U, P.pairs) + r : 0;
+        P.seg_range[2 * r + 1] = n > 0 ? pair_of_unit(u0 + n - 1, U, P.pairs) + r + 1 : 0;
+    }
+}
 __device__ __noinline__ void schedule(const Params &P, int pair, uint32_t rank, Ctrl *ctrl) {
     const int tid = threadIdx.x;
     bool bad = false;
+    if (tid == 0) {
+        ctrl->w_r0 = 0;
+        ctrl->w_pg0 = 0;
+    }
+    if (P.rows <= THREADS) {  // one pass: every row's length is read once, one block-wide scan
+        const int r = tid;
+        const int n = r < P.rows ? pages_of_row(P, r, bad) : 0;
+        long long U;
+        const long long u0 = block_scan(n, ctrl, U) - n;  // ends with a barrier (orders tid 0's defaults)
+        const long long s0 = unit_start(pair, U, P.pairs), s1 = unit_start(pair + 1, U, P.pairs);
+        if (tid == 0) ctrl->w_n = (int)(s1 - s0);
+        if (bad && pair == 0 && rank == 0) record_error(P.err, kErrBadSeqLen);
+        schedule_row(P, pair, rank, ctrl, r, n, u0, U, s0, s1);
+        __syncthreads();
+        return;
+    }
     long long U = 0;
     for (int base = 0; base < P.rows; base += THREADS) {  // pass 1: all units
         const int r = base + tid;
@@ -391,12 +434,7 @@ __device__ __noinline__ void schedule(const Params &P, int pair, uint32_t rank, 
     }
     if (bad && pair == 0 && rank == 0) record_error(P.err, kErrBadSeqLen);
     const long long s0 = unit_start(pair, U, P.pairs), s1 = unit_start(pair + 1, U, P.pairs);
-    if (tid == 0) {
-        ctrl->w_r0 = 0;
-        ctrl->w_pg0 = 0;
-        ctrl->w_n = (int)(s1 - s0);
-    }
-    __syncthreads();
+    if (tid == 0) ctrl->w_n = (int)(s1 - s0);
     long long carry = 0;
     for (int base = 0; base < P.rows; base += THREADS) {  // pass 2: locate s0, slot ranges
         const int r = base + tid;
@@ -404,25 +442,7 @@ __device__ __noinline__ void schedule(const Params &P, int pair, uint32_t rank, 
         const int n = r < P.rows ? pages_of_row(P, r, b2) : 0;
         long long chunk;
         const long long u0 = carry + block_scan(n, ctrl, chunk) - n;  // this row's first unit
-        if (n > 0 && u0 <= s0 && s0 < u0 + n) {  // the row holding unit s0
-            if (s1 > s0) {
-                ctrl->w_r0 = r;
-                ctrl->w_pg0 = (int)(s0 - u0);
-            } else if (rank == 0) {
-                // no units here, but this cluster's slot lies inside row r's slot range
-                for (int h = 0; h < NH; ++h) P.m_part[((size_t)pair + r) * NH + h] = -INFINITY;
-            }
-        }
-        if (pair == 0 && rank == 0 && r < P.rows) {
-            auto pair_of = [&](long long u) {  // the cluster holding unit u
-                int c = (int)(u * P.pairs / U);
-                while (c + 1 < P.pairs && unit_start(c + 1, U, P.pairs) <= u) ++c;
-                while (c > 0 && unit_start(c, U, P.pairs) > u) --c;
-                return c;
-            };
-            P.seg_range[2 * r] = n > 0 ? pair_of(u0) + r : 0;
-            P.seg_range[2 * r + 1] = n > 0 ? pair_of(u0 + n - 1) + r + 1 : 0;
-        }
+        schedule_row(P, pair, rank, ctrl, r, n, u0, U, s0, s1);
         carry += chunk;
     }
     __syncthreads();
@@ -505,6 +525,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
         mbar_init(bar(ctrl->o_free), 4);
         mbar_init(bar(ctrl->mma_idle[0]), 1);
         mbar_init(bar(ctrl->mma_idle[1]), 1);
+        mbar_init(bar(ctrl->never_done), 1);
         ctrl->abort = 0;
         ctrl->never = 0;
         if (rank == 1)
@@ -592,6 +613,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                     TRACE(1, u);
                 }
                 const int blk = block_of(P, it.r, it.pg);
+                // Test of the failure path: with copies (and soon MMAs) of the first page in flight,
+                // wait a short while on a barrier that nothing completes, and give up like any
+                // timed-out wait: abort flags in both CTAs, error word, bounded drains, exit.
+                if (P.test_give_up && u == 1 && !(ok = wait(bar(ctrl->never_done), 0u, abort_flag, 20000ull)))
+                    break;
                 if (!(ok = F8 ? load_f8(blk) : load(&tm_kv9, blk * PG))) break;
                 PROF_PAGE();
                 TRACE(2, u);
@@ -1463,6 +1489,7 @@ cudaError_t launch_decode_tc(const mla_dims_t &d, int B, int s_q, const void *q_
     P.l_part = w.l;
     P.scale_log2 = (float)(1.4426950408889634 / sqrt((double)(d.d_h + d.d_r)));
     P.err = err;
+    P.test_give_up = (d.flags & MLA_FLAG_TEST_GIVE_UP) ? 1 : 0;
     P.codes = f8 ? reinterpret_cast<const uint8_t *>(kv_pool) : nullptr;
     P.kv_scale = f8 ? kv_scale : nullptr;
     // The main and combine kernels are launched as programmatic dependents of the kernel before

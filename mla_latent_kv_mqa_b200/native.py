@@ -37,6 +37,7 @@ MLA_DTYPE_BF16 = 1
 MLA_DTYPE_FP8_E4M3 = 2
 MLA_FLAG_SIMT_DECODE = 1
 MLA_FLAG_SIMT_PROJ = 2
+MLA_FLAG_TEST_GIVE_UP = 4
 
 
 class MLAError(RuntimeError):

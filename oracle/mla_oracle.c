@@ -373,3 +373,15 @@ int mla_oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* Host threads for the following calls (the results do not depend on it: every (query, head)
+ * pair is computed by one thread in a fixed order).  For timing the oracle single-threaded. */
+void mla_oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

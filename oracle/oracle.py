@@ -70,6 +70,7 @@ def lib() -> ctypes.CDLL:
         L.mla_oracle_cache_row_elems.argtypes = [ci, ci]
         L.mla_oracle_cache_row_elems.restype = ci
         L.mla_oracle_num_threads.restype = ci
+        L.mla_oracle_set_num_threads.argtypes = [ci]
         _lib = L
     return _lib
 
@@ -84,6 +85,11 @@ def _f64(a) -> np.ndarray:
 
 def num_threads() -> int:
     return int(lib().mla_oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Host threads of the following oracle calls (results are independent of it)."""
+    lib().mla_oracle_set_num_threads(int(n))
 
 
 def rope(x, pos: float, base: float = 1e4) -> np.ndarray:
