@@ -259,7 +259,18 @@ def peaks_of():
         return 6650.0, 1590.0, "fallback"
 
 
-def measure(name, K, warmup, world, dev, clock_warmup_s, with_clock=True):
+STEP_CALLS = {True: "mla_cache_append, mla_absorb_q, mla_decode_project",
+              False: "mla_cache_append, mla_absorb_q, mla_decode, mla_out_proj"}
+
+
+def fused_applies(wl) -> bool:
+    """mla_decode_project runs its fused merge + projection kernel on this workload (the
+    tensor-core shape: 128 heads, d_h 128, d_c 512, d_R 64, page 64, bf16 activations)."""
+    d = wl.dims
+    return (d.n_h, d.d_h, d.d_c, d.d_r, d.page) == (128, 128, 512, 64, 64) and wl.act_dtype == "bf16"
+
+
+def measure(name, K, warmup, world, dev, clock_warmup_s, with_clock=True, separate=False):
     """Time one workload: K steps of the whole path (CUDA graph, L2 flushed before each step),
     K decode-only replays, K end-to-end steps from pinned host buffers.  Returns a dict (device
     times already reduced to the max over ranks) and the workload."""
@@ -285,13 +296,19 @@ def measure(name, K, warmup, world, dev, clock_warmup_s, with_clock=True):
     o = torch.empty((T, wl.dims.n_h, wl.dims.d_h), dtype=torch.float32, device=dev)
     L.workspace(B, s_q, run.max_seq_len)
     decode_launches = 2  # split-KV main kernel + log-sum-exp combine
-    launches_per_step = 1 + 1 + decode_launches + 1
+    fused = fused_applies(wl) and not separate
+    # append + absorb + (main + fused merge/projection | main + combine + out_proj)
+    launches_per_step = 1 + 1 + (2 if fused else decode_launches + 1)
 
     def step(_unused=None, tok=(tok_seq, tok_pos, c_new, k_new), qin=(run.q_c, run.q_r, run.q_pos), out=o):
         L.append(run.cache, tok[2], tok[3], tok[0], tok[1], run.block_table)
         L.absorb(qin[0], qin[1], qin[2], out=q_abs)
-        L.decode(run.cache, q_abs, run.block_table, run.seq_lens, s_q, run.max_seq_len, o_lat=o_lat, lse=lse)
-        L.out_proj(o_lat, "f32", out=out)
+        if fused:
+            L.decode_project(run.cache, q_abs, run.block_table, run.seq_lens, s_q, run.max_seq_len, "f32",
+                             o=out, o_lat=o_lat, lse=lse)
+        else:
+            L.decode(run.cache, q_abs, run.block_table, run.seq_lens, s_q, run.max_seq_len, o_lat=o_lat, lse=lse)
+            L.out_proj(o_lat, "f32", out=out)
 
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(device=dev)
@@ -386,7 +403,7 @@ def measure(name, K, warmup, world, dev, clock_warmup_s, with_clock=True):
     if N.mla_get_last_device_error() != 0:
         raise SystemExit(f"device error during the timed region ({name})")
     del g_step, g_dec, g_e2e
-    res = dict(step_ms=step_ms, dec_ms=dec_ms, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
+    res = dict(step_ms=step_ms, dec_ms=dec_ms, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, fused=fused,
                launches=(launches_per_step + decode_launches) * K, clocks=clk.summary() if with_clock else None)
     del run, flush, h_pack, d_pack, h_out
     torch.cuda.synchronize()
@@ -429,7 +446,7 @@ def run_mine(args):
         dist.barrier()
 
     K = args.steps
-    r, wl = measure(args.config, K, args.warmup, world, dev, args.clock_warmup_s)
+    r, wl = measure(args.config, K, args.warmup, world, dev, args.clock_warmup_s, separate=args.separate)
     rf = roofline_of(wl, r["dec_ms"])
     tokens = job_tokens(wl.T, world)
     line = None
@@ -442,7 +459,8 @@ def run_mine(args):
             "config": {"workload": WORKLOADS[args.config], "batch_per_gpu": wl.B, "s_q": wl.s_q,
                        "context": int(wl.seq_lens.max()), "parallelism": f"replicas x{world}",
                        "l2": "flushed before every timed step (512 MiB write outside the events)",
-                       "launch": "each step is one CUDA-graph replay of the four calls"},
+                       "launch": "each step is one CUDA-graph replay of the calls",
+                       "calls": STEP_CALLS[r["fused"]]},
             "decode": {"kernel": "mla_decode (tcgen05 split-KV main with in-kernel schedule + LSE combine)",
                        "ms": r["dec_ms"], "tokens_per_s": tokens / (r["dec_ms"] * 1e-3), "cache_gbs": rf["gbs"],
                        "tflops": rf["tfl"], "frac_hbm": rf["gbs"] / rf["hbm_peak"],
@@ -453,7 +471,7 @@ def run_mine(args):
                          "algorithmic_per_launch": rf["cache_bytes"] if rf["bound"] == "hbm" else rf["flops"]},
             "e2e": {"value": tokens / (r["e2e_ms"] * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"],
                     "d2h_bytes_per_step": r["d2h"], "ms_per_step": r["e2e_ms"],
-                    "how": "CUDA graph of one pinned H2D copy of the packed inputs + the four calls + D2H of o; host reads o each step"},
+                    "how": "CUDA graph of one pinned H2D copy of the packed inputs + the step's calls + D2H of o; host reads o each step"},
             "gpu_launches": r["launches"],
             "clocks": r["clocks"],
         }
@@ -468,10 +486,10 @@ def run_mine(args):
         for name in WORKLOADS:
             if name == args.config:
                 continue
-            r2, wl2 = measure(name, k2, args.warmup, world, dev, 0.8)
+            r2, wl2 = measure(name, k2, args.warmup, world, dev, 0.8, separate=args.separate)
             rf2 = roofline_of(wl2, r2["dec_ms"])
             t2 = job_tokens(wl2.T, world)
-            c = {"workload": WORKLOADS[name], "steps": k2, "step_ms": r2["step_ms"],
+            c = {"workload": WORKLOADS[name], "steps": k2, "step_ms": r2["step_ms"], "calls": STEP_CALLS[r2["fused"]],
                  "tokens_per_s": t2 / (r2["step_ms"] * 1e-3),
                  "decode_ms": r2["dec_ms"], "decode_tokens_per_s": t2 / (r2["dec_ms"] * 1e-3),
                  "cache_gbs": rf2["gbs"], "tflops": rf2["tfl"], "frac_hbm": rf2["gbs"] / rf2["hbm_peak"],
@@ -520,6 +538,8 @@ def main():
     ap.add_argument("--config", default="v3", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", action="store_true", help="time only --config (no per-workload block)")
+    ap.add_argument("--separate", action="store_true",
+                    help="step with mla_decode + mla_out_proj instead of mla_decode_project")
     ap.add_argument("--plain-steps", type=int, default=0, help="run N untimed eager steps and exit (profiling)")
     ap.add_argument("--batch", type=int, default=None, help="with --plain-steps: batch of the v3 or mtp_fp8 workload")
     args = ap.parse_args()

@@ -226,6 +226,61 @@ mla_status_t mla_decode_fixed_scratch(const mla_dims_t *dims, int B, int s_q, co
 mla_status_t mla_out_proj(const mla_dims_t *dims, int T, const float *o_lat, const void *w_uv,
                           void *o, mla_dtype_t out_dtype, mla_stream_t stream);
 
+/* ----------------------------------------------------------------------------------------
+ * mla_decode_project -- mla_decode followed by mla_out_proj in one call: the attention of
+ * mla_decode, then o = W^UV_h o_lat (행렬 흡수 section: the value up-projection applied after
+ * the aggregation).  Where the tensor-core kernels apply (n_h = 128, d_h = 128, d_c = 512,
+ * d_r = 64, page 64, bf16 activations, bf16 or FP8 cache, no MLA_FLAG_SIMT_* flag), the merge
+ * of the split partials and the projection run as ONE kernel, which never reads o_lat back;
+ * elsewhere the call runs mla_decode and mla_out_proj one after the other.  Either way o,
+ * o_lat and lse are bit for bit those of mla_decode followed by mla_out_proj.
+ *   Arguments as for mla_decode, plus
+ *   w_uv       [n_h*d_h, d_c] act dtype (as for mla_out_proj; written before the call)
+ *   o          [B*s_q, n_h, d_h] of out_dtype (F32 or BF16), written
+ *   o_lat      [B*s_q, n_h, d_c] fp32, written; 16-byte aligned
+ *   lse        as for mla_decode (may be NULL)
+ *   workspace  as for mla_decode (mla_decode_workspace_size)
+ * Errors: those of mla_decode and mla_out_proj; MLA_ERR_INVALID_ARG also for a null w_uv or
+ * o, or an o_lat that is not 16-byte aligned.
+ * ---------------------------------------------------------------------------------------- */
+mla_status_t mla_decode_project(const mla_dims_t *dims, int B, int s_q, const void *q_abs,
+                                const void *kv_pool, const void *kr_pool, const float *kv_scale,
+                                const int32_t *block_table, int max_blocks_per_seq, int num_blocks,
+                                const int32_t *seq_lens, int max_seq_len, void *workspace,
+                                size_t workspace_bytes, const void *w_uv, void *o,
+                                mla_dtype_t out_dtype, float *o_lat, float *lse,
+                                mla_stream_t stream);
+
+/* ----------------------------------------------------------------------------------------
+ * Sequence split across GPUs (long contexts): exact merge of decode results.
+ *
+ * MLA article, section 한계 (limitations): every head reads the whole latent cache, so tensor
+ * parallelism over heads cannot shard it.  The context can be split instead: each rank holds
+ * a contiguous range of every sequence's pages, runs mla_decode (s_q = 1) over its own pages
+ * only, and the ranks' results merge exactly.  For query row r and head h, with rank i's
+ * (o_lat_i, lse_i) from mla_decode:
+ *     M = max_i lse_i,  w_i = e^{lse_i - M},
+ *     o_lat = sum_i w_i o_lat_i / sum_i w_i,   lse = M + ln sum_i w_i.
+ * One step per rank before the cross-rank sum and one after it:
+ *   1. lse_max = all-reduce(max) of lse over the ranks       (the caller's collective)
+ *   2. mla_lse_merge_prepare: acc = [w o_lat ; w]            (this rank)
+ *   3. acc = all-reduce(sum) of acc over the ranks            (the caller's collective)
+ *   4. mla_lse_merge_finish: o_lat = acc_o / acc_w, lse = M + ln acc_w
+ * Arguments (device pointers, fp32, row-major):
+ *   o_lat   [rows, n_h, d_c]  this rank's mla_decode output (prepare) / the merged one (finish)
+ *   lse     [rows, n_h]       this rank's lse (prepare, natural log; -inf: no token) / merged
+ *                             (finish; may be NULL)
+ *   lse_max [rows, n_h]       the maximum of lse over the ranks
+ *   acc     [rows * n_h * (d_c + 1)]  w o_lat for every (row, head), then the rows*n_h weights
+ *                             w; the caller owns it and sums it over the ranks between the calls
+ * A row and head that no rank saw (every lse -inf) merge to o_lat = 0, lse = -inf.  Errors:
+ * MLA_ERR_INVALID_ARG for a negative or oversized count or a null pointer (rows = 0 is a no-op).
+ * ---------------------------------------------------------------------------------------- */
+mla_status_t mla_lse_merge_prepare(int rows, int n_h, int d_c, const float *o_lat, const float *lse,
+                                   const float *lse_max, float *acc, mla_stream_t stream);
+mla_status_t mla_lse_merge_finish(int rows, int n_h, int d_c, const float *acc, const float *lse_max,
+                                  float *o_lat, float *lse, mla_stream_t stream);
+
 /* Reads and clears the device error word of the current device.  Synchronises the device.
  * Returns MLA_OK, MLA_ERR_BAD_BLOCK_TABLE, MLA_ERR_BAD_SEQ_LEN or MLA_ERR_DEVICE_TIMEOUT
  * (the first condition seen since the last call), or MLA_ERR_CUDA. */

@@ -298,52 +298,6 @@ __device__ __forceinline__ float max32(const float (&x)[32]) {
     return fmaxf(fmaxf(a, b), fmaxf(c, d));
 }
 
-#ifdef MLA_TRACE
-// Development instrumentation: globaltimer stamps of pipeline events of one cluster.  Each warp
-// of each CTA writes its own 4096-entry region (no atomics on the traced path).
-constexpr int kTraceRegion = 4096;
-constexpr int kTraceMax = 2 * 16 * kTraceRegion;
-__device__ uint32_t g_trace[2 * kTraceMax];
-__device__ __forceinline__ void trace_event(int pair, uint32_t code, uint32_t unit, uint32_t &n) {
-    if (pair != MLA_TRACE) return;
-    const uint32_t region = cluster_ctarank() * 16 + (threadIdx.x >> 5);
-    if (n < kTraceRegion) {
-        const uint32_t i = region * kTraceRegion + n++;
-        g_trace[2 * i] = code | (unit << 8);
-        g_trace[2 * i + 1] = (uint32_t)globaltimer();
-    }
-}
-#define TRACE(code, unit) trace_event(pair, (code), (uint32_t)(unit), tr_n)
-#else
-#define TRACE(code, unit) ((void)0)
-#endif
-
-#ifdef MLA_SPAN
-// Development instrumentation: globaltimer stamps of the phases of every CTA of the last launch
-// (0 entry, 1 set up, 2 dependency wait done, 3 scheduled, 4 first S read, 5 last softmax done,
-// 6 last epilogue done, 7 exit).
-__device__ unsigned long long g_span[512][8];
-#define SPAN(i) (g_span[blockIdx.x & 511][i] = globaltimer())
-#else
-#define SPAN(i) ((void)0)
-#endif
-
-#ifdef MLA_PROF
-// Development instrumentation: per role and phase, clock cycles summed over a warp's pages
-// (lane 0), added once per warp into g_prof[rank][warp][phase] at the end; [..][..][7] counts pages.
-__device__ unsigned long long g_prof[2][16][8];
-#define PROF_DECL long long pf_acc[8] = {}; long long pf_t = clock64();
-#define PROF_MARK(i) do { const long long _n = clock64(); pf_acc[i] += _n - pf_t; pf_t = _n; } while (0)
-#define PROF_PAGE() (pf_acc[7] += 1)
-#define PROF_FLUSH() do { if (lane == 0) for (int _i = 0; _i < 8; ++_i) \
-    atomicAdd(&g_prof[cluster_ctarank()][warp][_i], (unsigned long long)pf_acc[_i]); } while (0)
-#else
-#define PROF_DECL
-#define PROF_MARK(i) ((void)0)
-#define PROF_PAGE() ((void)0)
-#define PROF_FLUSH() ((void)0)
-#endif
-
 // ---- the cluster's share of the work (every CTA computes it; cluster 0 also writes the
 // per-row slot ranges the combine kernel reads) --------------------------------------------
 // All (query row, page) units are numbered row by row; cluster c takes units
@@ -485,11 +439,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
     const uint32_t rank = cluster_ctarank();
     const int pair = blockIdx.x >> 1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) SPAN(0);
     warm_tables(P);
-#ifdef MLA_TRACE
-    uint32_t tr_n = 0;
-#endif
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < KV_STAGES; ++i) {
@@ -540,16 +490,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
     __syncthreads();
     tc_fence_after();
     cluster_sync();
-    if (threadIdx.x == 0) SPAN(1);
     // Everything above overlaps the kernel before this one; inputs are read from here on.
     pdl_trigger();
     pdl_wait();
-    if (threadIdx.x == 0) SPAN(2);
     schedule(P, pair, rank, ctrl);
-    if (threadIdx.x == 0) SPAN(3);
     const uint32_t tmem = ctrl->tmem_base;
     const uint32_t peer = rank ^ 1u;
-    if (threadIdx.x == 0) TRACE(20 + rank, (uint32_t)clock64() >> 8);
     auto fail = [&]() {
         if (*abort_flag == 0) {
             *abort_flag = 1;
@@ -573,13 +519,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             uint32_t nph[KV_STAGES] = {};
             int u = 0;
             bool ok = true;
-            PROF_DECL
             auto load = [&](const CUtensorMap *map, int y) -> bool {
                 if (!wait(bar(ctrl->kv_empty[st.i]), st.ph ^ 1u, abort_flag)) return false;
-                PROF_MARK(0);
                 mbar_arrive_expect_tx(bar(ctrl->kv_full[st.i]), KV_STAGE);
                 tma_load_3d(data_s + st.i * KV_STAGE, map, 0, y, 0, bar(ctrl->kv_full[st.i]));
-                PROF_MARK(1);
                 issued[st.i] = 1;
                 nph[st.i] = st.ph;
                 st.adv(KVS);
@@ -610,7 +553,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             while (ok && !it.done()) {
                 if (it.first) {
                     if (!(ok = load(&tm_q9, it.r * NH) && load(&tm_q9, it.r * NH + 64))) break;
-                    TRACE(1, u);
                 }
                 const int blk = block_of(P, it.r, it.pg);
                 // Test of the failure path: with copies (and soon MMAs) of the first page in flight,
@@ -619,13 +561,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 if (P.test_give_up && u == 1 && !(ok = wait(bar(ctrl->never_done), 0u, abort_flag, 20000ull)))
                     break;
                 if (!(ok = F8 ? load_f8(blk) : load(&tm_kv9, blk * PG))) break;
-                PROF_PAGE();
-                TRACE(2, u);
                 ++u;
                 it.next(P);
             }
             if (!ok) fail();
-            PROF_FLUSH();
             for (int i = 0; i < KV_STAGES; ++i)  // drain: every copy this thread started has landed
                 if (issued[i]) wait(bar(ctrl->kv_full[i]), nph[i], never);
             for (int i = 0; i < 2; ++i)
@@ -650,19 +589,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             uint32_t cv_ph = 0;  // FP8: phase bit of conv_full[i] (it completes on page uses only)
             int u = 0;
             bool ok = true, any = false;
-            PROF_DECL
             while (ok && !it.done()) {
                 if (it.first) {
                     st.adv(KVS, 2);  // the segment's Q stages (copied to TMEM by the softmax warps)
-                    PROF_MARK(4);
                     if (!(ok = wait(bar(ctrl->q_ready), qn & 1u, abort_flag))) break;
-                    PROF_MARK(0);
                     ++qn;
                 }
-                PROF_MARK(4);
                 if (!(ok = wait(bar(ctrl->s_free[sb.i]), sb.ph ^ 1u, abort_flag))) break;
                 if (part && !(ok = wait(bar(ctrl->k0_done[sb.i]), sb.ph, abort_flag))) break;
-                PROF_MARK(1);
                 tc_fence_after();  // orders the MMAs after the softmax's TMEM zeroing / thread 0's MMAs
                 // TMA-filled shared memory needs no tcgen05 fence: the mbarrier completion already
                 // makes it visible to MMAs issued after the wait.
@@ -671,8 +605,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                     if (!(ok = wait(bar(ctrl->conv_full[st.i]), (cv_ph >> st.i) & 1u, abort_flag))) break;
                     cv_ph ^= 1u << st.i;
                 }
-                PROF_MARK(2);
-                TRACE(6 + part, u);
                 const uint32_t d = tmem + S_COL + sb.i * PG;
                 const uint32_t kvb = data_s + st.i * KV_STAGE;
 #pragma unroll 1
@@ -688,17 +620,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 }
                 mma_commit(bar(ctrl->kv_empty[st.i]));
                 mma_commit(bar(ctrl->s_full[sb.i]));
-                PROF_MARK(3);
-                PROF_PAGE();
                 any = true;
-                TRACE(3 + part, u);
                 ++u;
                 st.adv(KVS);
                 sb.adv(S_SETS);
                 it.next(P);
             }
             if (!ok) fail();
-            PROF_FLUSH();
             if (any) {  // drain: the MMAs this thread issued are complete before TMEM is released
                 mma_commit(bar(ctrl->mma_idle[part]));
                 wait(bar(ctrl->mma_idle[part]), 0u, never);
@@ -791,21 +719,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 tmem_wait_st();
             }
             if (!it.done()) ok = load_q() && first_page();  // load_q's barrier also orders the zeroing before q_ready
-            PROF_DECL
             while (ok && !it.done()) {
                 if (F8 && !it.last()) {  // the next page of this segment (its stage follows this page's)
                     Ring c = st;
                     c.adv(KVS);
                     if (!(ok = convert(c))) break;
-                    PROF_MARK(6);
                 }
-                if (t == 0) TRACE(27, u);
-                if (t == 32) TRACE(67, u);
                 bool good = wait(bar(ctrl->s_full[sb.i]), sb.ph, abort_flag);
-                if (t == 0 && u == 0) SPAN(4);
-                PROF_MARK(0);
-                if (t == 0) TRACE(5, u);
-                if (t == 32) TRACE(45, u);
                 float mine[32], other[32];
                 {
                     uint32_t a[32], b[32];
@@ -820,12 +740,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                         other[j] = __uint_as_float(b[j]);
                     }
                 }
-                if (t == 0) TRACE(26, u);
-                if (t == 32) TRACE(66, u);
                 const uint32_t s_buf = sb.i;  // zeroed and released after the vote (all warps have read it)
-                PROF_MARK(1);
-                if (t == 0) TRACE(24, u);
-                if (t == 32) TRACE(64, u);
                 sb.adv(S_SETS);
                 st.adv(KVS);  // this page's stage
 
@@ -861,21 +776,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 }
                 l = l * fac + (s0 + s1);
                 m_used = m_new;
-                PROF_MARK(2);
-                if (t == 0) TRACE(25, u);
-                if (t == 32) TRACE(65, u);
                 if (last && half) ctrl->lx[seg & 1][h] = l;  // read by the other half after the vote
 
                 // ---- hand P to the senders through TMEM (one buffer: the senders took the last) ----
                 good = good && wait(bar(ctrl->p_taken), (uint32_t)(u & 1) ^ 1u, abort_flag);
-                PROF_MARK(3);
-                if (t == 0) TRACE(28, u);
                 if (named_red_or(!good, BAR_FAIL, SM_THREADS)) {
                     ok = false;
                     break;
                 }
-                PROF_MARK(4);
-                if (t == 0) TRACE(29, u);
                 tc_fence_after();
                 {   // every softmax warp has read this S buffer: zero my half for its next page
                     uint32_t z[32];
@@ -892,9 +800,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                     mbar_arrive(bar(ctrl->s_free[s_buf]));
                     mbar_arrive(bar(ctrl->p_ready));
                 }
-                PROF_MARK(5);
-                PROF_PAGE();
-                if (t == 0) TRACE(30, u);
                 ++u;
 
                 if (last) {
@@ -909,13 +814,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                     // The last page's S is complete, so every QK MMA of this segment has finished
                     // and the next segment's Q may overwrite TMEM now.
                     if (it.left > 1 && !(ok = load_q() && first_page())) break;
-                    PROF_MARK(6);
                 }
                 it.next(P);
             }
             if (!ok) fail();
-            if (t == 0) SPAN(5);
-            PROF_FLUSH();
         } else if (warp >= SD_WARP0 && warp < SD_WARP0 + 4) {  // senders: P in TMEM -> CTA 1 slot
             const int t = threadIdx.x - SD_WARP0 * 32;          // 0..127
             const int quarter = warp & 3;
@@ -928,18 +830,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             int u = 0;
             bool ok = true;
             uint32_t sent = 0, sent_ph = 0;  // slots with a message out, and its phase
-            PROF_DECL
             while (ok && !it.done()) {
                 bool good = wait(bar(ctrl->p_ready), (uint32_t)(u & 1), abort_flag);
-                PROF_MARK(0);
                 good = good && wait<true>(bar(ctrl->pfree[ps.i]), ps.ph ^ 1u, abort_flag);
-                PROF_MARK(5);
                 if (named_red_or(!good, BAR_SFAIL, SD_THREADS)) {
                     ok = false;
                     break;
                 }
-                PROF_MARK(1);
-                if (t == 0) TRACE(9, u);
                 tc_fence_after();
                 uint32_t pv[32];
                 tmem_ld32(tmem + lane_base + P_COL, pv);
@@ -948,29 +845,23 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(ctrl->p_taken));
-                PROF_MARK(2);
                 const uint32_t slot = slot_r + ps.i * P_SLOT, fb = p_full_r + ps.i * 8;
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
                     st_async_v4(slot + h * 128 + ((c ^ (h & 7)) << 4), pv[4 * c], pv[4 * c + 1], pv[4 * c + 2],
                                 pv[4 * c + 3], fb);
                 st_async_b32(slot + P_FACT + h * 4, __float_as_uint(fac), fb);
-                PROF_MARK(3);
                 const bool any = named_red_or(fac != 1.f, BAR_SFLAG, SD_THREADS);
                 if (t == 0) {
                     st_async_b32(slot + P_FLAG, any ? 1u : 0u, fb);
                     sent |= 1u << ps.i;
                     sent_ph = (sent_ph & ~(1u << ps.i)) | (ps.ph << ps.i);
-                    TRACE(8, u);
                 }
-                PROF_MARK(4);
-                PROF_PAGE();
                 ps.adv(P_SLOTS);
                 ++u;
                 it.next(P);
             }
             if (!ok) fail();
-            PROF_FLUSH();
             // drain: CTA 1's arrivals on our slot barriers (its MMA commits, its readers) for the
             // messages still out have landed before this CTA can leave
             if (t == 0)
@@ -989,7 +880,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             for (int i = 0; i < VH_STAGES; ++i) issued[i] = 0;
             int u = 0;
             bool ok = true;
-            PROF_DECL
             Ring vg{0, 0};  // FP8: staging slot of the next half page of raw codes
             int g_issued[2] = {0, 0};
             uint32_t g_nph[2] = {0u, 0u};
@@ -1006,9 +896,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                     vg.adv(2);
                 }
                 for (int hh = 0; !F8 && hh < 2; ++hh) {
-                    PROF_MARK(1);
                     if (!(ok = wait(bar(ctrl->v_empty[vs.i]), vs.ph ^ 1u, abort_flag))) break;
-                    PROF_MARK(0);
                     mbar_arrive_expect_tx(bar(ctrl->v_full[vs.i]), VH_STAGE);
                     tma_load_3d(data_s + V_OFF + vs.i * VH_STAGE, &tm_kv4, 0, blk * PG, hh * 4,
                                 bar(ctrl->v_full[vs.i]));
@@ -1017,13 +905,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                     vs.adv(VH_STAGES);
                 }
                 if (!ok) break;
-                PROF_PAGE();
-                TRACE(11, u);
                 ++u;
                 it.next(P);
             }
             if (!ok) fail();
-            PROF_FLUSH();
             for (int i = 0; i < VH_STAGES; ++i)
                 if (issued[i]) wait(bar(ctrl->v_full[i]), nph[i], never);
             for (int i = 0; i < 2; ++i)
@@ -1037,12 +922,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             uint32_t vr_ph = 0;  // phase bit of v_ready[i]: it completes only on ragged pages
             int u = 0;
             bool ok = true, any = false;
-            PROF_DECL
             while (ok && !it.done()) {
-                PROF_MARK(4);
                 if (!(ok = wait<true>(bar(ctrl->p_full[ps.i]), ps.ph, abort_flag))) break;
-                PROF_MARK(0);
-                TRACE(13, u);
                 const uint32_t pa = data_s + P_OFF + ps.i * P_SLOT;
                 const uint32_t flag = ld_shared_u32(pa + P_FLAG);
                 mbar_arrive_expect_tx(bar(ctrl->p_full[ps.i]), MSG_BYTES);  // arm the slot's next use
@@ -1054,9 +935,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 if (first && nseg > 0) {
                     if (!(ok = wait(bar(ctrl->o_free), (nseg - 1) & 1u, abort_flag))) break;
                 }
-                PROF_MARK(1);
                 for (int nh = 0; nh < 2; ++nh) {
-                    PROF_MARK(3);
                     if (ragged) {
                         ok = wait(bar(ctrl->v_ready[vs.i]), (vr_ph >> vs.i) & 1u, abort_flag);
                         vr_ph ^= 1u << vs.i;
@@ -1064,8 +943,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                         ok = wait(bar(ctrl->v_full[vs.i]), vs.ph, abort_flag);
                     }
                     if (!ok) break;
-                    PROF_MARK(2);
-                    if (nh == 0) TRACE(12, u);
                     tc_fence_after();
                     const uint32_t vb = data_s + V_OFF + vs.i * VH_STAGE;
 #pragma unroll
@@ -1080,17 +957,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 if (!ok) break;
                 mma_commit(bar(ctrl->pv_done[ps.i]));
                 mma_commit_mc(bar(ctrl->pfree[ps.i]), (uint16_t)1u);  // CTA 0's slot barrier
-                PROF_MARK(3);
-                PROF_PAGE();
                 any = true;
-                TRACE(14, u);
                 ++u;
                 if (it.last()) ++nseg;
                 ps.adv(P_SLOTS);
                 it.next(P);
             }
             if (!ok) fail();
-            PROF_FLUSH();
             if (any) {
                 mma_commit(bar(ctrl->mma_idle[0]));
                 wait(bar(ctrl->mma_idle[0]), 0u, never);
@@ -1107,13 +980,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             it.init(P, &ctrl->w_r0);
             Ring vs{0, 0}, vg{0, 0};
             bool ok = true;
-            PROF_DECL
             while (ok && !it.done()) {
                 for (int hh = 0; hh < 2; ++hh) {
                     bool w = wait(bar(ctrl->vstg_full[vg.i]), vg.ph, abort_flag);
-                    PROF_MARK(0);
                     w = w && wait(bar(ctrl->v_empty[vs.i]), vs.ph ^ 1u, abort_flag);
-                    PROF_MARK(1);
                     if (named_red_or(!w, BAR_VCONV, VC_THREADS)) {
                         ok = false;
                         break;
@@ -1133,15 +1003,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                         mbar_arrive(bar(ctrl->v_full[vs.i]));
                         mbar_arrive(bar(ctrl->vstg_empty[vg.i]));
                     }
-                    PROF_MARK(2);
                     vs.adv(VH_STAGES);
                     vg.adv(2);
                 }
-                PROF_PAGE();
                 it.next(P);
             }
             if (!ok && lane == 0) fail();
-            PROF_FLUSH();
         } else if (warp >= EP_WARP0 && warp < EP_WARP0 + 4) {  // ragged zeroing, rescale, epilogue
             const int quarter = warp & 3;
             const int h = quarter * 32 + lane;
@@ -1152,7 +1019,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             Ring vs{0, 0}, ps{0, 0}, prev{0, 0};
             int u = 0;
             bool ok = true;
-            PROF_DECL
             while (ok && !it.done()) {
                 const int valid = it.valid();
                 // 1. ragged last page: zero token rows [valid, 64) of both V halves
@@ -1174,7 +1040,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                     }
                     if (!ok) break;
                 }
-                PROF_MARK(0);
                 // 2. the P message: this head's factor and the flag; then free the slot for reading
                 if (!(ok = __all_sync(0xffffffffu, wait<true>(bar(ctrl->p_full[ps.i]), ps.ph, abort_flag)))) break;
                 const uint32_t pa = data_s + P_OFF + ps.i * P_SLOT;
@@ -1182,8 +1047,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 const uint32_t flag = ld_shared_u32(pa + P_FLAG);
                 __syncwarp();
                 if (lane == 0) mbar_arrive_remote(pfree_r + ps.i * 8);
-                PROF_MARK(1);
-                if (h == 0) TRACE(16, u);
                 const bool last = it.last();
                 // 3. lazy rescale of O rows whose running max moved (the previous page's PV done)
                 if (flag) {
@@ -1205,13 +1068,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(ctrl->corr_done));
                 }
-                PROF_MARK(2);
                 // 4. end of segment: this warp writes its 32 heads of the partial O (not normalised)
                 // as bf16 pairs of columns, [slot][d_c / 2][n_h] words, so that each store
                 // instruction of the warp covers one whole 128-byte line (32 heads, one pair).
                 if (last) {
                     if (!(ok = __all_sync(0xffffffffu, wait(bar(ctrl->pv_done[ps.i]), ps.ph, abort_flag)))) break;
-                    if (h == 0) TRACE(18, u);
                     tc_fence_after();
                     uint32_t *dst = P.o_part + (size_t)(pair + it.r) * (DC / 2) * NH + h;
 #pragma unroll 1
@@ -1227,11 +1088,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(ctrl->o_free));
-                    if (h == 0) TRACE(19, u);
-                    if (h == 0) SPAN(6);
                 }
-                PROF_MARK(3);
-                PROF_PAGE();
                 ++u;
                 prev = ps;
                 vs.adv(VH_STAGES, 2);
@@ -1239,14 +1096,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 it.next(P);
             }
             if (!ok && lane == 0) fail();
-            PROF_FLUSH();
         }
     }
 
     // ---- teardown: both CTAs quiesce before either releases TMEM or exits ----
     __syncwarp();
-    if (threadIdx.x == 0) TRACE(22 + rank, (uint32_t)clock64() >> 8);
-    if (threadIdx.x == 0) SPAN(7);
     tc_fence_before();
     __syncthreads();
     cluster_sync();
@@ -1411,38 +1265,6 @@ size_t tc_layout(int pairs, int rows, char *base, TcWs *w) {
 
 }  // namespace
 
-#ifdef MLA_TRACE
-// Copies the whole trace buffer (kTraceMax entries of {code | unit << 8, time}) and clears it.
-extern "C" int mla_trace_dump(uint32_t *host, int max_entries) {
-    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
-    const int n = max_entries < kTraceMax ? max_entries : kTraceMax;
-    cudaMemcpyFromSymbol(host, g_trace, 2 * (size_t)n * sizeof(uint32_t));
-    static uint32_t zeros[2 * kTraceMax];
-    cudaMemcpyToSymbol(g_trace, zeros, sizeof(zeros));
-    return n;
-}
-#endif
-
-#ifdef MLA_SPAN
-// Copies the phase stamps (512 x 8 u64) of the last launch.
-extern "C" int mla_span_dump(unsigned long long *host) {
-    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
-    cudaMemcpyFromSymbol(host, g_span, sizeof(g_span));
-    return 0;
-}
-#endif
-
-#ifdef MLA_PROF
-// Copies the phase accumulators (2 x 16 x 8 u64) and clears them.
-extern "C" int mla_prof_dump(unsigned long long *host) {
-    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
-    cudaMemcpyFromSymbol(host, g_prof, sizeof(g_prof));
-    static unsigned long long zeros[2 * 16 * 8];
-    cudaMemcpyToSymbol(g_prof, zeros, sizeof(zeros));
-    return 0;
-}
-#endif
-
 bool tc_supported(const mla_dims_t &d) {
     return d.n_h == NH && d.d_c == DC && d.d_r == ROW - DC && d.page_size == PG &&
            d.act_dtype == MLA_DTYPE_BF16 && (d.kv_dtype == MLA_DTYPE_BF16 || d.kv_dtype == MLA_DTYPE_FP8_E4M3);
@@ -1457,7 +1279,8 @@ size_t tc_workspace_bytes(const mla_dims_t &d, int B, int s_q, int) {
 cudaError_t launch_decode_tc(const mla_dims_t &d, int B, int s_q, const void *q_abs,
                              const void *kv_pool, const void *kr_pool, const float *kv_scale, const int32_t *bt,
                              int max_blocks, int num_blocks, const int32_t *seq_lens, int max_seq_len,
-                             void *ws, size_t ws_bytes, float *o_lat, float *lse, cudaStream_t st) {
+                             void *ws, size_t ws_bytes, float *o_lat, float *lse, cudaStream_t st,
+                             const FusedOutProj *fuse) {
     const int rows = B * s_q;
     const bool f8 = d.kv_dtype == MLA_DTYPE_FP8_E4M3;
     const int pairs = tc_pairs(d);
@@ -1512,6 +1335,9 @@ cudaError_t launch_decode_tc(const mla_dims_t &d, int B, int s_q, const void *q_
     e = f8 ? cudaLaunchKernelEx(&cfg, decode_tc_kernel<true>, tm_kv9, tm_kv4, tm_q9, P)
            : cudaLaunchKernelEx(&cfg, decode_tc_kernel<false>, tm_kv9, tm_kv4, tm_q9, P);
     if (e != cudaSuccess) return e;
+    if (fuse)
+        return launch_combine_out_proj_tc(d, rows, w.seg_range, w.o, w.m, w.l, o_lat, lse, fuse->w_uv, fuse->o,
+                                          fuse->out_dtype, st);
     const int vec_out = (reinterpret_cast<uintptr_t>(o_lat) & 15) == 0;
     cfg.gridDim = dim3(rows, DC / CMB_COLS);
     cfg.blockDim = dim3(NH);

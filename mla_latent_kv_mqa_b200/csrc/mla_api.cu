@@ -151,11 +151,14 @@ size_t mla_decode_workspace_size(const mla_dims_t *dims, int B, int s_q, int max
     return simt_workspace_bytes(*dims, B, s_q, max_seq_len);
 }
 
-mla_status_t mla_decode(const mla_dims_t *dims, int B, int s_q, const void *q_abs,
-                        const void *kv_pool, const void *kr_pool, const float *kv_scale,
-                        const int32_t *block_table, int max_blocks_per_seq, int num_blocks,
-                        const int32_t *seq_lens, int max_seq_len, void *workspace,
-                        size_t workspace_bytes, float *o_lat, float *lse, mla_stream_t stream) {
+// mla_decode and mla_decode_project: `fuse` (may be null) routes the merge of the split
+// partials through the fused combine + output projection kernel.
+static mla_status_t decode_impl(const mla_dims_t *dims, int B, int s_q, const void *q_abs,
+                                const void *kv_pool, const void *kr_pool, const float *kv_scale,
+                                const int32_t *block_table, int max_blocks_per_seq, int num_blocks,
+                                const int32_t *seq_lens, int max_seq_len, void *workspace,
+                                size_t workspace_bytes, float *o_lat, float *lse, mla_stream_t stream,
+                                const FusedOutProj *fuse) {
     mla_status_t s = check_dims(dims);
     if (s != MLA_OK) return s;
     if (B < 0 || s_q < 1 || max_blocks_per_seq < 1 || num_blocks < 1 || max_seq_len < 1)
@@ -182,11 +185,48 @@ mla_status_t mla_decode(const mla_dims_t *dims, int B, int s_q, const void *q_ab
             return MLA_ERR_INVALID_ARG;
         return from_cuda(launch_decode_tc(*dims, B, s_q, q_abs, kv_pool, kr_pool, kv_scale,
                                           block_table, max_blocks_per_seq, num_blocks, seq_lens,
-                                          max_seq_len, workspace, workspace_bytes, o_lat, lse, st));
+                                          max_seq_len, workspace, workspace_bytes, o_lat, lse, st, fuse));
     }
+    if (fuse) return MLA_ERR_UNSUPPORTED;  // callers fuse only where the tensor-core path applies
     return from_cuda(launch_decode_simt(*dims, B, s_q, q_abs, kv_pool, kr_pool, kv_scale,
                                         block_table, max_blocks_per_seq, num_blocks, seq_lens,
                                         max_seq_len, workspace, o_lat, lse, st));
+}
+
+mla_status_t mla_decode(const mla_dims_t *dims, int B, int s_q, const void *q_abs,
+                        const void *kv_pool, const void *kr_pool, const float *kv_scale,
+                        const int32_t *block_table, int max_blocks_per_seq, int num_blocks,
+                        const int32_t *seq_lens, int max_seq_len, void *workspace,
+                        size_t workspace_bytes, float *o_lat, float *lse, mla_stream_t stream) {
+    return decode_impl(dims, B, s_q, q_abs, kv_pool, kr_pool, kv_scale, block_table, max_blocks_per_seq,
+                       num_blocks, seq_lens, max_seq_len, workspace, workspace_bytes, o_lat, lse, stream,
+                       nullptr);
+}
+
+mla_status_t mla_decode_project(const mla_dims_t *dims, int B, int s_q, const void *q_abs,
+                                const void *kv_pool, const void *kr_pool, const float *kv_scale,
+                                const int32_t *block_table, int max_blocks_per_seq, int num_blocks,
+                                const int32_t *seq_lens, int max_seq_len, void *workspace,
+                                size_t workspace_bytes, const void *w_uv, void *o,
+                                mla_dtype_t out_dtype, float *o_lat, float *lse,
+                                mla_stream_t stream) {
+    mla_status_t s = check_dims(dims);
+    if (s != MLA_OK) return s;
+    if (B < 0 || s_q < 1) return MLA_ERR_INVALID_ARG;
+    if (B == 0) return MLA_OK;
+    if (!w_uv || !o || !o_lat || !aligned(o_lat, 16)) return MLA_ERR_INVALID_ARG;
+    if (!act_ok(out_dtype)) return MLA_ERR_UNSUPPORTED;
+    if ((int64_t)B * s_q > INT_MAX) return MLA_ERR_INVALID_ARG;
+    if (use_tc(dims) && proj_tc_supported(*dims) && !(dims->flags & MLA_FLAG_SIMT_PROJ)) {
+        const FusedOutProj fuse{w_uv, o, out_dtype};
+        return decode_impl(dims, B, s_q, q_abs, kv_pool, kr_pool, kv_scale, block_table, max_blocks_per_seq,
+                           num_blocks, seq_lens, max_seq_len, workspace, workspace_bytes, o_lat, lse, stream,
+                           &fuse);
+    }
+    s = decode_impl(dims, B, s_q, q_abs, kv_pool, kr_pool, kv_scale, block_table, max_blocks_per_seq,
+                    num_blocks, seq_lens, max_seq_len, workspace, workspace_bytes, o_lat, lse, stream, nullptr);
+    if (s != MLA_OK) return s;
+    return mla_out_proj(dims, B * s_q, o_lat, w_uv, o, out_dtype, stream);
 }
 
 // mla_decode on the library's fixed scratch array instead of a caller workspace.  The size
@@ -205,6 +245,22 @@ mla_status_t mla_decode_fixed_scratch(const mla_dims_t *dims, int B, int s_q, co
     return mla_decode(dims, B, s_q, q_abs, kv_pool, kr_pool, kv_scale, block_table,
                       max_blocks_per_seq, num_blocks, seq_lens, max_seq_len, scratch,
                       kDecodeScratchBytes, o_lat, lse, stream);
+}
+
+mla_status_t mla_lse_merge_prepare(int rows, int n_h, int d_c, const float *o_lat, const float *lse,
+                                   const float *lse_max, float *acc, mla_stream_t stream) {
+    if (rows < 0 || n_h < 1 || d_c < 1 || (int64_t)rows * n_h > INT_MAX) return MLA_ERR_INVALID_ARG;
+    if (rows == 0) return MLA_OK;
+    if (!o_lat || !lse || !lse_max || !acc) return MLA_ERR_INVALID_ARG;
+    return from_cuda(launch_lse_merge_prepare(rows, n_h, d_c, o_lat, lse, lse_max, acc, (cudaStream_t)stream));
+}
+
+mla_status_t mla_lse_merge_finish(int rows, int n_h, int d_c, const float *acc, const float *lse_max,
+                                  float *o_lat, float *lse, mla_stream_t stream) {
+    if (rows < 0 || n_h < 1 || d_c < 1 || (int64_t)rows * n_h > INT_MAX) return MLA_ERR_INVALID_ARG;
+    if (rows == 0) return MLA_OK;
+    if (!acc || !lse_max || !o_lat) return MLA_ERR_INVALID_ARG;
+    return from_cuda(launch_lse_merge_finish(rows, n_h, d_c, acc, lse_max, o_lat, lse, (cudaStream_t)stream));
 }
 
 mla_status_t mla_out_proj(const mla_dims_t *dims, int T, const float *o_lat, const void *w_uv,

@@ -110,14 +110,34 @@ cudaError_t launch_decode_simt(const mla_dims_t &d, int B, int s_q, const void *
 cudaError_t launch_combine(int rows, int n_h, int d_c, Partials p, const int32_t *seg_range,
                            int uniform, float *o_lat, float *lse, cudaStream_t st);
 
-// Tensor-core (tcgen05) decode for the DeepSeek-V3 shape.
+// Tensor-core (tcgen05) decode for the DeepSeek-V3 shape.  With `fuse`, the split partials
+// are merged by the fused combine + output projection kernel instead of the combine kernel.
+struct FusedOutProj {
+    const void *w_uv;
+    void *o;
+    mla_dtype_t out_dtype;
+};
 bool tc_supported(const mla_dims_t &d);
 size_t tc_workspace_bytes(const mla_dims_t &d, int B, int s_q, int max_seq_len);
 cudaError_t launch_decode_tc(const mla_dims_t &d, int B, int s_q, const void *q_abs,
                              const void *kv_pool, const void *kr_pool, const float *kv_scale,
                              const int32_t *bt, int max_blocks, int num_blocks,
                              const int32_t *seq_lens, int max_seq_len, void *ws,
-                             size_t ws_bytes, float *o_lat, float *lse, cudaStream_t st);
+                             size_t ws_bytes, float *o_lat, float *lse, cudaStream_t st,
+                             const FusedOutProj *fuse = nullptr);
+// The fused kernel: partials in the tensor-core decode's layout ([slot][d_c / 2][n_h] bf16
+// pairs, m and l per slot and head, per-row slot ranges) -> o_lat, lse (either may be null)
+// and o = W^UV_h o_lat.  o_lat, when given, must be 16-byte aligned.
+cudaError_t launch_combine_out_proj_tc(const mla_dims_t &d, int T, const int32_t *seg_range,
+                                       const uint32_t *o_part, const float *m_part, const float *l_part,
+                                       float *o_lat, float *lse, const void *w_uv, void *o,
+                                       mla_dtype_t out_dtype, cudaStream_t st);
+
+// Sequence split across GPUs: the per-rank steps of the exact log-sum-exp merge.
+cudaError_t launch_lse_merge_prepare(int rows, int n_h, int d_c, const float *o_lat, const float *lse,
+                                     const float *lse_max, float *acc, cudaStream_t st);
+cudaError_t launch_lse_merge_finish(int rows, int n_h, int d_c, const float *acc, const float *lse_max,
+                                    float *o_lat, float *lse, cudaStream_t st);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

@@ -35,25 +35,11 @@ constexpr int NWB = DCL / 64;       // 8 boxes per head
 struct __align__(8) ProjCtrl {
     uint64_t a_full[NWB];
     uint64_t b_done[2];
+    uint64_t b_full;  // fused combine: every column block of the B tile has arrived
     uint64_t d_full;
     uint32_t tmem_base;
     uint32_t abort;
 };
-
-#ifdef MLA_PROF
-// Development instrumentation: per CTA of the last launch of each kernel (0 = absorb,
-// 1 = out_proj), globaltimer at entry and exit and clock64 offsets from entry at marks 1..13.
-__device__ unsigned long long g_proj_prof[2][512][16];
-#define PPROF_DECL(kid) const long long pp_c0 = clock64(); const int pp_k = (kid); \
-    unsigned long long *pp_row = g_proj_prof[pp_k][min(blockIdx.x + blockIdx.y * gridDim.x, 511u)]; \
-    if (threadIdx.x == 0) pp_row[0] = globaltimer();
-#define PPROF_MARK(i) do { if (threadIdx.x == 0) pp_row[i] = clock64() - pp_c0; } while (0)
-#define PPROF_END() do { if (threadIdx.x == 0) { pp_row[15] = globaltimer(); pp_row[14] = clock64() - pp_c0; } } while (0)
-#else
-#define PPROF_DECL(kid)
-#define PPROF_MARK(i)
-#define PPROF_END()
-#endif
 
 // ------------------------------------------------------------------------------------------
 // out_proj: smem = W_h (8 x 16 KB, K-major) + the CTA's o_lat tokens as bf16 hi + lo, one
@@ -74,7 +60,6 @@ template <typename To>
 __global__ void __launch_bounds__(128, 1)
 out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int n_h, const float *__restrict__ o_lat,
                    To *__restrict__ o, unsigned *err) {
-    PPROF_DECL(1)
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_u32(smem_raw);
     const uint32_t data_s = (raw_s + 1023u) & ~1023u;
@@ -103,10 +88,8 @@ out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int n_h, con
         tmem_alloc(smem_u32(&ctrl->tmem_base), TNO);
         tmem_relinquish();
     }
-    PPROF_MARK(1);
     pdl_trigger();
     pdl_wait();  // o_lat is the previous kernel's output
-    PPROF_MARK(2);
     const uint32_t bs = data_s + OP_B;
     for (int idx = tid; idx < npad * 64; idx += 128) {
         const int r = idx >> 6, g = idx & 63, c = g & 7;
@@ -121,7 +104,6 @@ out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int n_h, con
         }
     }
     cp_async_wait_all();
-    PPROF_MARK(3);
     for (int idx = tid; idx < npad * 64; idx += 128) {
         const int r = idx >> 6, g = idx & 63, c = g & 7;
         const uint32_t hs = bs + (g >> 3) * OP_BBLK + r * 128 + ((c ^ (r & 7)) << 4);
@@ -145,7 +127,6 @@ out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int n_h, con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctrl->tmem_base;
-    PPROF_MARK(4);
     if (tid == 0) {
         const uint32_t idesc = idesc_bf16(128, npad, false, false);
         bool good = true;
@@ -165,11 +146,9 @@ out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int n_h, con
         }
         if (good) mma_commit(smem_u32(&ctrl->d_full));
         else *abort_flag = 1;
-        PPROF_MARK(5);
     }
     bool ok = __syncthreads_and(*abort_flag == 0);
     if (ok) ok = __syncthreads_and(wait(smem_u32(&ctrl->d_full), 0, abort_flag));
-    PPROF_MARK(6);
     if (ok) {
         tc_fence_after();
         const int d = warp * 32 + lane;
@@ -182,14 +161,192 @@ out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int n_h, con
     } else if (tid == 0) {
         record_error(err, kErrTimeout);
     }
-    PPROF_MARK(7);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, TNO);
     }
-    PPROF_END();
+}
+
+// ------------------------------------------------------------------------------------------
+// combine + out_proj in one kernel, after the tensor-core decode.
+// The decode leaves, per split slot s of a query row, the unnormalised partial O_s as bf16
+// pairs of columns laid out [slot][d_c / 2][n_h] words, with its log2-domain max m_s and sum
+// l_s per head.  The merge is the combine kernel's, term for term (same order, same fused
+// multiply-adds), so o_lat and lse come out bit-identical to it:
+//     M = max_s m_s,  w_s = 2^(m_s - M),  L = sum_s w_s l_s,
+//     o_lat = sum_s w_s O_s / L,  lse = (M + log2 L) ln 2.
+// Grid (n_h, tiles of TNO rows) in clusters of 8 CTAs along the heads.  CTA q of the cluster
+// that owns heads 8g..8g+7 merges column block q (64 latent columns) for all 8 heads and all
+// rows of its tile: a warp's loads then read 8 heads x 4 bytes = one whole 32-byte sector per
+// column pair, where a CTA merging only its own head would use 4 bytes of every sector it
+// reads.  The merged values go, split into bf16 hi + lo exactly as out_proj splits o_lat,
+// straight into the B tile of the CTA that owns the head (st.async into a peer's shared
+// memory, completing on its b_full barrier; a plain store for the CTA's own head); o_lat and
+// lse are also written out.  Then every CTA runs
+// the out_proj MMAs of its head as out_proj_tc_kernel does.
+// ------------------------------------------------------------------------------------------
+constexpr int CO_CLUSTER = 8;
+
+template <typename To>
+__global__ void __cluster_dims__(CO_CLUSTER, 1, 1) __launch_bounds__(128, 1)
+combine_out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int n_h,
+                           const int32_t *__restrict__ seg_range, const uint32_t *__restrict__ o_part,
+                           const float *__restrict__ m_part, const float *__restrict__ l_part,
+                           float *__restrict__ o_lat, float *__restrict__ lse, To *__restrict__ o,
+                           unsigned *err) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = smem_u32(smem_raw);
+    const uint32_t data_s = (raw_s + 1023u) & ~1023u;
+    ProjCtrl *ctrl = reinterpret_cast<ProjCtrl *>(smem_raw + (data_s - raw_s) + OP_DATA);
+    volatile uint32_t *abort_flag = &ctrl->abort;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h = blockIdx.x, t0 = blockIdx.y * TNO;
+    const int nt = min(TNO, T - t0);
+    const int npad = (nt + 15) & ~15;
+    const uint32_t q = cluster_ctarank();  // column block merged here; == h % 8
+    const int hg = h - (int)q;             // first head of the cluster
+
+    if (tid == 0) {
+        for (int i = 0; i < NWB; ++i) mbar_init(smem_u32(&ctrl->a_full[i]), 1);
+        mbar_init(smem_u32(&ctrl->b_full), 1);
+        mbar_init(smem_u32(&ctrl->d_full), 1);
+        ctrl->abort = 0;
+        // the 7 column blocks merged by the other CTAs of the cluster: nt rows x (hi + lo) x 128 B
+        mbar_arrive_expect_tx(smem_u32(&ctrl->b_full), (uint32_t)((CO_CLUSTER - 1) * nt * 256));
+        fence_mbarrier_init_cluster();
+        prefetch_tensormap(&tm_w);
+        for (int kb = 0; kb < NWB; ++kb) {
+            mbar_arrive_expect_tx(smem_u32(&ctrl->a_full[kb]), WBOX);
+            tma_load_2d(data_s + OP_A + kb * WBOX, &tm_w, kb * 64, h * DH, smem_u32(&ctrl->a_full[kb]));
+        }
+    }
+    if (warp == 0) {
+        __syncwarp();
+        tmem_alloc(smem_u32(&ctrl->tmem_base), TNO);
+        tmem_relinquish();
+    }
+    cluster_sync();  // every b_full of the cluster is initialised and armed before any st.async
+    pdl_trigger();
+    pdl_wait();      // the partials and the slot ranges are the decode's output
+    const uint32_t bs = data_s + OP_B;
+
+    // ---- merge: thread = (head i of the cluster, 8-column chunk c of block q, row parity) ----
+    {
+        const int i = tid & 7, c = (tid >> 3) & 7;
+        const int hh = hg + i;
+        const size_t slot_words = (size_t)(DCL / 2) * n_h;
+        const uint32_t *src = o_part + (size_t)(q * 32 + c * 4) * n_h + hh;
+        const uint32_t dst_bar = mapa(smem_u32(&ctrl->b_full), (uint32_t)i);
+        for (int r = tid >> 6; r < nt; r += 2) {
+            const int row = t0 + r;
+            const int s0 = __ldcg(seg_range + 2 * row), s1 = __ldcg(seg_range + 2 * row + 1);
+            float M = -INFINITY, L = 0.f, acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+            for (int s = s0; s < s1; ++s) M = fmaxf(M, __ldcg(m_part + (size_t)s * n_h + hh));
+            for (int s = s0; s < s1; ++s) {
+                const float ms = __ldcg(m_part + (size_t)s * n_h + hh);
+                if (ms == -INFINITY) continue;  // empty slot: weight 0, partials never written
+                const float w = exp2f(ms - M);
+                L = fmaf(w, __ldcg(l_part + (size_t)s * n_h + hh), L);
+                uint32_t v[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) v[k] = __ldcg(src + (size_t)s * slot_words + (size_t)k * n_h);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    acc[2 * k] = fmaf(w, __uint_as_float(v[k] << 16), acc[2 * k]);
+                    acc[2 * k + 1] = fmaf(w, __uint_as_float(v[k] & 0xffff0000u), acc[2 * k + 1]);
+                }
+            }
+            const float inv = L > 0.f ? 1.f / L : 0.f;
+            float x[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) x[j] = acc[j] * inv;
+            if (o_lat) {
+                float4 *dst = reinterpret_cast<float4 *>(o_lat + ((size_t)row * n_h + hh) * DCL + q * 64 + c * 8);
+                dst[0] = make_float4(x[0], x[1], x[2], x[3]);
+                dst[1] = make_float4(x[4], x[5], x[6], x[7]);
+            }
+            if (lse && q == 0 && c == 0)
+                lse[(size_t)row * n_h + hh] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const __nv_bfloat162 hv = __floats2bfloat162_rn(x[2 * k], x[2 * k + 1]);
+                const float2 hf = __bfloat1622float2(hv);
+                const __nv_bfloat162 lv = __floats2bfloat162_rn(x[2 * k] - hf.x, x[2 * k + 1] - hf.y);
+                hw[k] = *reinterpret_cast<const uint32_t *>(&hv);
+                lw[k] = *reinterpret_cast<const uint32_t *>(&lv);
+            }
+            const uint32_t loc = bs + q * OP_BBLK + r * 128 + ((c ^ (r & 7)) << 4);
+            if (i == (int)q) {  // this CTA's own head: a plain shared-memory store
+                st_shared_v4(loc, hw[0], hw[1], hw[2], hw[3]);
+                st_shared_v4(loc + TNO * 128, lw[0], lw[1], lw[2], lw[3]);
+            } else {
+                const uint32_t dst = mapa(loc, (uint32_t)i);
+                st_async_v4(dst, hw[0], hw[1], hw[2], hw[3], dst_bar);
+                st_async_v4(dst + TNO * 128, lw[0], lw[1], lw[2], lw[3], dst_bar);
+            }
+        }
+    }
+    // rows nt..npad-1 of the MMA's N are zero (only rows < nt are merged)
+    for (int idx = tid; idx < (npad - nt) * 64; idx += 128) {
+        const int r = nt + (idx >> 6), g = idx & 63, c = g & 7;
+        const uint32_t hs = bs + (g >> 3) * OP_BBLK + r * 128 + ((c ^ (r & 7)) << 4);
+        st_shared_v4(hs, 0u, 0u, 0u, 0u);
+        st_shared_v4(hs + TNO * 128, 0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctrl->tmem_base;
+    if (tid == 0) {
+        const uint32_t idesc = idesc_bf16(128, npad, false, false);
+        bool good = wait<true>(smem_u32(&ctrl->b_full), 0, abort_flag);
+        tc_fence_after();
+        for (int kb = 0; good && kb < NWB; ++kb) {
+            if (!wait(smem_u32(&ctrl->a_full[kb]), 0, abort_flag)) {
+                good = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t bhi = bs + kb * OP_BBLK, blo = bhi + TNO * 128;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint64_t a = sdesc_sw128(data_s + OP_A + kb * WBOX + k * 32, 16, 1024);
+                mma_ss(tmem, a, sdesc_sw128(bhi + k * 32, 16, 1024), idesc, (kb | k) != 0 ? 1u : 0u);
+                mma_ss(tmem, a, sdesc_sw128(blo + k * 32, 16, 1024), idesc, 1u);
+            }
+        }
+        if (good) mma_commit(smem_u32(&ctrl->d_full));
+        else *abort_flag = 1;
+    }
+    bool ok = __syncthreads_and(*abort_flag == 0);
+    if (ok) ok = __syncthreads_and(wait(smem_u32(&ctrl->d_full), 0, abort_flag));
+    if (ok) {
+        tc_fence_after();
+        const int d = warp * 32 + lane;
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16), v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (j < nt) o[((size_t)(t0 + j) * n_h + h) * DH + d] = from_f32<To>(__uint_as_float(v[j]));
+    } else if (tid == 0) {
+        record_error(err, kErrTimeout);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TNO);
+    }
+    // No CTA leaves while a peer may still be sending into its shared memory: every CTA has
+    // issued its sends and waited for its own tile before it reaches this barrier.
+    cluster_sync();
 }
 
 // ------------------------------------------------------------------------------------------
@@ -206,7 +363,6 @@ __global__ void __launch_bounds__(128, 1)
 absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int n_h, const __grid_constant__ RopeFreqs rope,
                  const __nv_bfloat16 *__restrict__ q_c, const __nv_bfloat16 *__restrict__ q_r,
                  const int32_t *__restrict__ pos, __nv_bfloat16 *__restrict__ q_abs, unsigned *err) {
-    PPROF_DECL(0)
     pdl_trigger();  // the decode that follows may set itself up (it waits for q_abs on the device)
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_u32(smem_raw);
@@ -237,9 +393,7 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int n_h, const
         tmem_alloc(smem_u32(&ctrl->tmem_base), 512);
         tmem_relinquish();
     }
-    PPROF_MARK(1);
     pdl_wait();  // the queries may be the previous kernel's output
-    PPROF_MARK(2);
     // q_c rows of this head for the tile's tokens -> two K-major column blocks (k 0-63, 64-127),
     // copied asynchronously so that the RoPE loads below go out at the same time.
     const uint32_t bq = data_s + AB_B;
@@ -278,7 +432,6 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int n_h, const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctrl->tmem_base;
-    PPROF_MARK(3);
     if (tid == 0) {
         const uint32_t idesc = idesc_bf16(128, npad, true, false);
         bool good = true;
@@ -296,11 +449,9 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int n_h, const
         }
         if (good) mma_commit(smem_u32(&ctrl->d_full));
         else *abort_flag = 1;
-        PPROF_MARK(4);
     }
     bool ok = __syncthreads_and(*abort_flag == 0);
     if (ok) ok = __syncthreads_and(wait(smem_u32(&ctrl->d_full), 0, abort_flag));
-    PPROF_MARK(6);
     if (ok) {
         // D[c, t] (lane = latent column) -> bf16 rows [t][d_c] in the (now free) weight region,
         // then whole-row 16-byte stores.
@@ -334,14 +485,12 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int n_h, const
     } else if (tid == 0) {
         record_error(err, kErrTimeout);
     }
-    PPROF_MARK(7);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
-    PPROF_END();
 }
 
 }  // namespace
@@ -398,15 +547,21 @@ cudaError_t launch_out_proj_tc(const mla_dims_t &d, int T, const float *o_lat, c
                             reinterpret_cast<float *>(o), device_error_word());
 }
 
-#ifdef MLA_PROF
-// Copies the per-CTA timelines (2 x 512 x 16 u64) of the projection kernels and clears them.
-extern "C" int mla_proj_prof_dump(unsigned long long *host) {
-    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
-    cudaMemcpyFromSymbol(host, g_proj_prof, sizeof(g_proj_prof));
-    static unsigned long long zeros[2 * 512 * 16];
-    cudaMemcpyToSymbol(g_proj_prof, zeros, sizeof(zeros));
-    return 0;
+cudaError_t launch_combine_out_proj_tc(const mla_dims_t &d, int T, const int32_t *seg_range,
+                                       const uint32_t *o_part, const float *m_part, const float *l_part,
+                                       float *o_lat, float *lse, const void *w_uv, void *o,
+                                       mla_dtype_t out_dtype, cudaStream_t st) {
+    if (d.n_h % CO_CLUSTER != 0) return cudaErrorInvalidValue;
+    CUtensorMap tm;
+    if (!tmap_bf16_2d(&tm, w_uv, DCL, (uint64_t)d.n_h * DH, DCL * 2, 64, 128)) return cudaErrorInvalidValue;
+    const dim3 grid(d.n_h, (T + TNO - 1) / TNO);
+    if (out_dtype == MLA_DTYPE_BF16)
+        return launch_dependent(combine_out_proj_tc_kernel<__nv_bfloat16>, grid, OP_SMEM, st, tm, T, d.n_h,
+                                seg_range, o_part, m_part, l_part, o_lat, lse,
+                                reinterpret_cast<__nv_bfloat16 *>(o), device_error_word());
+    return launch_dependent(combine_out_proj_tc_kernel<float>, grid, OP_SMEM, st, tm, T, d.n_h, seg_range,
+                            o_part, m_part, l_part, o_lat, lse, reinterpret_cast<float *>(o),
+                            device_error_word());
 }
-#endif
 
 }  // namespace mla

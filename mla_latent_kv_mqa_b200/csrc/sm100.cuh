@@ -91,16 +91,7 @@ template <bool kCluster = false>
 __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort,
                                      uint64_t limit_ns = 2000000000ull) {
     if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
-#ifdef MLA_WAIT_INLINE
-    const uint64_t t0 = globaltimer();
-    while (true) {
-        if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
-        if (*abort) return false;
-        if (globaltimer() - t0 > limit_ns) return false;
-    }
-#else
     return wait_poll<kCluster>(bar, parity, abort, limit_ns);
-#endif
 }
 
 // ---- programmatic dependent launch ----------------------------------------------------------

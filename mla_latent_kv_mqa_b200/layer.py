@@ -112,6 +112,25 @@ class MLADecodeLayer:
                      lse, stream)
         return o_lat, lse
 
+    def decode_project(self, cache: PagedLatentCache, q_abs, block_table, seq_lens, s_q, max_seq_len,
+                       out_dtype="f32", o=None, o_lat=None, lse=None, stream=None):
+        """decode followed by out_proj in one library call; returns (o, o_lat, lse)."""
+        d = self.dims
+        B, max_blocks = block_table.shape
+        rows = B * s_q
+        dt = DTYPE[out_dtype]
+        if o is None:
+            o = torch.empty((rows, d.n_h, d.d_h), dtype=TORCH_ACT[dt], device=self.device)
+        if o_lat is None:
+            o_lat = torch.empty((rows, d.n_h, d.d_c), dtype=torch.float32, device=self.device)
+        if lse is None:
+            lse = torch.empty((rows, d.n_h), dtype=torch.float32, device=self.device)
+        ws = self.workspace(B, s_q, max_seq_len)
+        N.mla_decode_project(d, B, s_q, q_abs, cache.kv_pool, cache.kr_pool, cache.kv_scale, block_table,
+                             max_blocks, cache.num_blocks, seq_lens, max_seq_len, ws, ws.numel(), self.w_uv,
+                             o, dt, o_lat, lse, stream)
+        return o, o_lat, lse
+
     def out_proj(self, o_lat, out_dtype="f32", out=None, stream=None):
         d = self.dims
         T = o_lat.shape[0]

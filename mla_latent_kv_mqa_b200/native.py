@@ -68,12 +68,17 @@ _lib.mla_decode.argtypes = [_dp, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _
 _lib.mla_decode_fixed_scratch.argtypes = [_dp, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _i,
                                           _vp, _vp, _vp]
 _lib.mla_out_proj.argtypes = [_dp, _i, _vp, _vp, _vp, _i, _vp]
+_lib.mla_decode_project.argtypes = [_dp, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _i, _vp, _sz,
+                                    _vp, _vp, _i, _vp, _vp, _vp]
+_lib.mla_lse_merge_prepare.argtypes = [_i, _i, _i, _vp, _vp, _vp, _vp, _vp]
+_lib.mla_lse_merge_finish.argtypes = [_i, _i, _i, _vp, _vp, _vp, _vp, _vp]
 _lib.mla_get_last_device_error.argtypes = []
 _lib.mla_status_string.argtypes = [_i]
 _lib.mla_status_string.restype = ctypes.c_char_p
 _lib.mla_version.restype = _i
 for _f in ("mla_absorb_q", "mla_cache_append", "mla_decode", "mla_decode_fixed_scratch", "mla_out_proj",
-           "mla_get_last_device_error"):
+           "mla_decode_project", "mla_get_last_device_error", "mla_lse_merge_prepare",
+           "mla_lse_merge_finish"):
     getattr(_lib, _f).restype = _i
 
 
@@ -158,6 +163,27 @@ def mla_decode_fixed_scratch(dims, B, s_q, q_abs, kv_pool, kr_pool, kv_scale, bl
 def mla_out_proj(dims, T, o_lat, w_uv, o, out_dtype=MLA_DTYPE_F32, stream=None):
     _check(_lib.mla_out_proj(ctypes.byref(dims), T, _ptr(o_lat), _ptr(w_uv), _ptr(o), out_dtype,
                              _stream(stream)), "mla_out_proj")
+
+
+def mla_decode_project(dims, B, s_q, q_abs, kv_pool, kr_pool, kv_scale, block_table, max_blocks_per_seq,
+                       num_blocks, seq_lens, max_seq_len, workspace, workspace_bytes, w_uv, o, out_dtype,
+                       o_lat, lse=None, stream=None):
+    """mla_decode followed by mla_out_proj (one fused merge + projection kernel where it applies)."""
+    _check(_lib.mla_decode_project(ctypes.byref(dims), B, s_q, _ptr(q_abs), _ptr(kv_pool), _ptr(kr_pool),
+                                   _ptr(kv_scale), _ptr(block_table), max_blocks_per_seq, num_blocks,
+                                   _ptr(seq_lens), max_seq_len, _ptr(workspace), workspace_bytes, _ptr(w_uv),
+                                   _ptr(o), out_dtype, _ptr(o_lat), _ptr(lse), _stream(stream)),
+           "mla_decode_project")
+
+
+def mla_lse_merge_prepare(rows, n_h, d_c, o_lat, lse, lse_max, acc, stream=None):
+    _check(_lib.mla_lse_merge_prepare(rows, n_h, d_c, _ptr(o_lat), _ptr(lse), _ptr(lse_max), _ptr(acc),
+                                      _stream(stream)), "mla_lse_merge_prepare")
+
+
+def mla_lse_merge_finish(rows, n_h, d_c, acc, lse_max, o_lat, lse=None, stream=None):
+    _check(_lib.mla_lse_merge_finish(rows, n_h, d_c, _ptr(acc), _ptr(lse_max), _ptr(o_lat), _ptr(lse),
+                                     _stream(stream)), "mla_lse_merge_finish")
 
 
 def mla_get_last_device_error() -> int:

@@ -77,6 +77,25 @@ def test_host_argument_checks(N):
     assert L.mla_decode(*args) == N.MLA_ERR_INVALID_ARG
     assert N.mla_decode_workspace_size(simt, 1 << 20, 1 << 12, 4096) == 0
     assert L.mla_cache_append(dp, 1, 8, 8, 8, 8, 8, 1, 1 << 26, 1, 8, None, None, None) == N.MLA_ERR_INVALID_ARG
+    # decode + projection: the decode's checks, plus w_uv, o, and a 16-byte aligned o_lat
+    def dp_call(w_uv=16, o=16, out_dtype=0, o_lat=16, q_abs=16, B=2):
+        return L.mla_decode_project(dp, B, 1, q_abs, 16, None, None, 16, 4, 8, 16, 256, 256, 1 << 30,
+                                    w_uv, o, out_dtype, o_lat, 16, None)
+    assert dp_call(w_uv=None) == N.MLA_ERR_INVALID_ARG
+    assert dp_call(o=None) == N.MLA_ERR_INVALID_ARG
+    assert dp_call(o_lat=None) == N.MLA_ERR_INVALID_ARG
+    assert dp_call(o_lat=8) == N.MLA_ERR_INVALID_ARG
+    assert dp_call(q_abs=None) == N.MLA_ERR_INVALID_ARG
+    assert dp_call(out_dtype=N.MLA_DTYPE_FP8_E4M3) == N.MLA_ERR_UNSUPPORTED
+    assert dp_call(B=0, w_uv=None) == N.MLA_OK
+    # sequence-split merge: sizes, null pointers with work to do, (rows, n_h) within int
+    for f in (L.mla_lse_merge_prepare, L.mla_lse_merge_finish):
+        for rows, n_h, d_c in [(-1, 1, 1), (1, 0, 1), (1, 1, 0), (1 << 20, 1 << 12, 8)]:
+            assert f(rows, n_h, d_c, 16, 16, 16, 16, None) == N.MLA_ERR_INVALID_ARG
+        assert f(0, 1, 1, None, None, None, None, None) == N.MLA_OK
+    assert L.mla_lse_merge_prepare(1, 1, 1, None, 16, 16, 16, None) == N.MLA_ERR_INVALID_ARG
+    assert L.mla_lse_merge_prepare(1, 1, 1, 16, 16, 16, None, None) == N.MLA_ERR_INVALID_ARG
+    assert L.mla_lse_merge_finish(1, 1, 1, 16, 16, None, 16, None) == N.MLA_ERR_INVALID_ARG
 
 
 def test_workspace_size_is_positive_and_monotone(N):
