@@ -40,6 +40,9 @@ WORKLOADS = {
     "long": "V3 dims, batch 4, context 131072, per-token norms LogNormal(0,0.5), bf16",
     "mtp_fp8": "V3 dims, batch 128, context 8192, s_q=2 causal, FP8 e4m3 content + bf16 RoPE key",
 }
+PREFILL = ("MHA-mode prefill (mla_prefill, K/V reconstructed from the latent): V3 dims n_h=128, d_h=128, "
+           "d_c=512, d_R=64, bf16, 4 prompts x 4096 tokens, causal")
+PREFILL_LENS = [4096] * 4
 FLUSH_BYTES = 512 << 20
 # DRAM bytes (read + write) per launch of the main decode kernel, from one ncu capture of the
 # same workload and build (`ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum -k
@@ -270,7 +273,7 @@ def fused_applies(wl) -> bool:
     return (d.n_h, d.d_h, d.d_c, d.d_r, d.page) == (128, 128, 512, 64, 64) and wl.act_dtype == "bf16"
 
 
-def measure(name, K, warmup, world, dev, clock_warmup_s, with_clock=True, separate=False):
+def measure(name, K, warmup, world, dev, clock_warmup_s, with_clock=True, project=False):
     """Time one workload: K steps of the whole path (CUDA graph, L2 flushed before each step),
     K decode-only replays, K end-to-end steps from pinned host buffers.  Returns a dict (device
     times already reduced to the max over ranks) and the workload."""
@@ -296,7 +299,7 @@ def measure(name, K, warmup, world, dev, clock_warmup_s, with_clock=True, separa
     o = torch.empty((T, wl.dims.n_h, wl.dims.d_h), dtype=torch.float32, device=dev)
     L.workspace(B, s_q, run.max_seq_len)
     decode_launches = 2  # split-KV main kernel + log-sum-exp combine
-    fused = fused_applies(wl) and not separate
+    fused = fused_applies(wl) and project
     # append + absorb + (main + fused merge/projection | main + combine + out_proj)
     launches_per_step = 1 + 1 + (2 if fused else decode_launches + 1)
 
@@ -411,6 +414,88 @@ def measure(name, K, warmup, world, dev, clock_warmup_s, with_clock=True, separa
     return res, wl
 
 
+def prefill_flops(wl):
+    """FLOPs of one mla_prefill by the method's definition: the K and V reconstruction
+    (2 T d_c n_h d_h each) and the causal attention (per head and visible (query, key) pair,
+    2 (d_h + d_R) for the score and 2 d_h for the value sum)."""
+    d = wl.dims
+    L = wl.seq_lens.astype(np.int64)
+    pairs = int((L * (L + 1) // 2).sum())
+    attn = pairs * d.n_h * 2 * ((d.d_h + d.d_r) + d.d_h)
+    up = 2 * 2 * wl.T * d.d_c * d.n_h * d.d_h
+    return attn, up
+
+
+def measure_prefill(K, warmup, dev, with_clock=True, lens=None):
+    """K timed mla_prefill calls (CUDA graph of the one call, L2 flushed before each)."""
+    import torch
+    from mla_latent_kv_mqa_b200 import native as N
+    from mla_latent_kv_mqa_b200 import workloads as W
+    from tests.harness import PrefillRun
+    wl = W.make_prefill(9, lens or PREFILL_LENS, name="prefill")
+    run = PrefillRun(wl, dev)
+    o = torch.empty((wl.T, wl.dims.n_h, wl.dims.d_h), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((wl.T, wl.dims.n_h), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    call = lambda: run.layer.prefill(run.q_c, run.q_r, run.c_kv, run.k_r, run.cu, run.max_len, o=o, lse=lse)
+    with torch.cuda.stream(stream):
+        for _ in range(max(warmup, 3)):
+            flush.fill_(1)
+            call()
+        stream.synchronize()
+        if N.mla_get_last_device_error() != 0:
+            raise SystemExit("device error during the prefill warm-up")
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            call()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        bus = torch.cuda.get_device_properties(dev).pci_bus_id
+        with ClockSampler(bus if with_clock else -1) as clk:
+            t_end = time.time() + 0.8
+            while time.time() < t_end:
+                g.replay()
+                stream.synchronize()
+            t_timed = time.time()
+            for k in range(K):
+                flush.fill_(k & 0xFF)
+                ev[k][0].record(stream)
+                g.replay()
+                ev[k][1].record(stream)
+            stream.synchronize()
+            clk.window = (t_timed - 0.5, time.time() + 0.15)
+            time.sleep(0.15)
+    ms = sum(a.elapsed_time(b) for a, b in ev) / K
+    if N.mla_get_last_device_error() != 0:
+        raise SystemExit("device error during the timed prefill")
+    del g
+    res = dict(ms=ms, launches=3 * K, clocks=clk.summary() if with_clock else None)
+    del run, flush, o, lse
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res, wl
+
+
+def prefill_cpu_baseline(wl, budget_s: float = 8.0):
+    """The fp64 naive-mode oracle, as it stands, on sampled prompt rows (all heads; rows drawn
+    uniformly over the prompts' positions, so the mean cost per row is the workload's) until
+    ``budget_s`` is spent."""
+    from oracle import oracle as orc
+    from tests.harness import prefill_oracle_rows
+    orc.build()
+    rng = np.random.default_rng(0)
+    t0 = time.perf_counter()
+    n = 0
+    while time.perf_counter() - t0 < budget_s:
+        b = int(rng.integers(0, wl.B))
+        t = int(rng.integers(0, wl.seq_lens[b]))
+        prefill_oracle_rows(wl, orc, [(b, t)], np.arange(wl.dims.n_h))
+        n += 1
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": orc.num_threads(), "kind": "oracle",
+            "sample": f"{n} prompt rows drawn uniformly, all {wl.dims.n_h} heads, fp64 naive mode, {dt:.1f} s"}
+
+
 def roofline_of(wl, dec_ms):
     hbm_peak, tc_peak, src = peaks_of()
     cache_bytes, flops = algorithmic(wl)
@@ -446,7 +531,7 @@ def run_mine(args):
         dist.barrier()
 
     K = args.steps
-    r, wl = measure(args.config, K, args.warmup, world, dev, args.clock_warmup_s, separate=args.separate)
+    r, wl = measure(args.config, K, args.warmup, world, dev, args.clock_warmup_s, project=args.project)
     rf = roofline_of(wl, r["dec_ms"])
     tokens = job_tokens(wl.T, world)
     line = None
@@ -486,7 +571,7 @@ def run_mine(args):
         for name in WORKLOADS:
             if name == args.config:
                 continue
-            r2, wl2 = measure(name, k2, args.warmup, world, dev, 0.8, separate=args.separate)
+            r2, wl2 = measure(name, k2, args.warmup, world, dev, 0.8, project=args.project)
             rf2 = roofline_of(wl2, r2["dec_ms"])
             t2 = job_tokens(wl2.T, world)
             c = {"workload": WORKLOADS[name], "steps": k2, "step_ms": r2["step_ms"], "calls": STEP_CALLS[r2["fused"]],
@@ -506,6 +591,21 @@ def run_mine(args):
                 c["cpu_baseline"] = cpu_baseline(wl2)
             configs[name] = c
             del wl2
+        # the MHA-mode prefill (a second workload of the library, not a decode step)
+        rp, wlp = measure_prefill(k2, args.warmup, dev)
+        attn, up = prefill_flops(wlp)
+        hbm_peak, tc_peak, src = peaks_of()
+        tfl = (attn + up) / (rp["ms"] * 1e-3) / 1e12
+        c = {"workload": PREFILL, "steps": k2, "ms": rp["ms"], "tokens_per_s": wlp.T / (rp["ms"] * 1e-3),
+             "tflops": tfl, "flops": {"attention": attn, "kv_reconstruction": up},
+             "roofline": {"bound": "tensor", "achieved": tfl, "peak": tc_peak, "unit": "TFLOP/s",
+                          "frac": tfl / tc_peak, "peak_source": src,
+                          "note": "whole call (prep + K/V GEMM + attention) against the dense bf16 peak"},
+             "gpu_launches": rp["launches"], "clocks": rp["clocks"]}
+        if not args.no_cpu_baseline:
+            c["cpu_baseline"] = prefill_cpu_baseline(wlp)
+        configs["prefill"] = c
+        del wlp
         line["configs"] = configs
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -523,7 +623,11 @@ def run_plain(args):
     run = GpuRun(wl)
     run.fill_cache()
     for _ in range(args.plain_steps):
-        run.step()
+        if args.plain_project:
+            q_abs = run.layer.absorb(run.q_c, run.q_r, run.q_pos)
+            run.layer.decode_project(run.cache, q_abs, run.block_table, run.seq_lens, wl.s_q, run.max_seq_len, "f32")
+        else:
+            run.step()
     torch.cuda.synchronize()
     print(f"plain steps done: {args.plain_steps} x {wl.name}")
 
@@ -538,11 +642,28 @@ def main():
     ap.add_argument("--config", default="v3", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", action="store_true", help="time only --config (no per-workload block)")
-    ap.add_argument("--separate", action="store_true",
-                    help="step with mla_decode + mla_out_proj instead of mla_decode_project")
+    ap.add_argument("--prefill-only", action="store_true", help="time only the MHA-mode prefill workload")
+    ap.add_argument("--prefill-lens", default=None, help="with --prefill-only: comma-separated prompt lengths")
+    ap.add_argument("--plain-project", action="store_true",
+                    help="with --plain-steps: steps through mla_decode_project")
+    ap.add_argument("--project", action="store_true",
+                    help="step with mla_decode_project (fused merge + projection) instead of mla_decode + "
+                         "mla_out_proj")
     ap.add_argument("--plain-steps", type=int, default=0, help="run N untimed eager steps and exit (profiling)")
     ap.add_argument("--batch", type=int, default=None, help="with --plain-steps: batch of the v3 or mtp_fp8 workload")
     args = ap.parse_args()
+    if args.prefill_only:
+        import torch
+        from mla_latent_kv_mqa_b200 import build
+        build.build()
+        torch.cuda.set_device(0)
+        lens = [int(x) for x in args.prefill_lens.split(",")] if args.prefill_lens else None
+        rp, wlp = measure_prefill(args.steps, args.warmup, torch.device("cuda", 0), lens=lens)
+        attn, up = prefill_flops(wlp)
+        print(json.dumps({"workload": PREFILL if lens is None else f"prefill, prompts {lens}",
+                          "ms": rp["ms"], "tokens_per_s": wlp.T / (rp["ms"] * 1e-3),
+                          "tflops": (attn + up) / (rp["ms"] * 1e-3) / 1e12, "clocks": rp["clocks"]}), flush=True)
+        return
     if args.plain_steps:
         run_plain(args)
     elif args.impl == "reference":

@@ -252,6 +252,41 @@ mla_status_t mla_decode_project(const mla_dims_t *dims, int B, int s_q, const vo
                                 mla_stream_t stream);
 
 /* ----------------------------------------------------------------------------------------
+ * mla_prefill -- causal attention over whole prompts in MHA ("naive") mode: the keys and
+ * values are reconstructed per head from the latent (구조 section), k_{j,h} = [W^UK_h c_j ;
+ * RoPE(k^R_j, j)] and v_{j,h} = W^UV_h c_j, and for every prompt token t and head h
+ *     o[t,h,:] = sum_{j <= t} softmax_j( [q^C ; RoPE(q^R, t)]_{t,h} . k_{j,h} / sqrt(d_h + d_r) ) v_{j,h}
+ * (분리 RoPE section output equation).  The 한계 section and the mode remarks of the 행렬 흡수
+ * section: with as many queries as keys, reconstructing K and V once costs less than the
+ * 576-wide latent scores of the absorbed form, which pays off in decode only.
+ * Positions are token indices within each prompt (0 .. L_b - 1).  The call does not write the
+ * cache: append the prompt with mla_cache_append for the decode steps that follow.
+ * Supported shape: d_h = 128, d_c = 512, d_r = 64, even n_h, bf16 activations and weights
+ * (MLA_ERR_UNSUPPORTED otherwise).  Precision: bf16 operands (K and V rounded to bf16 once,
+ * P to bf16), fp32 accumulation and softmax.
+ *   B            number of prompts
+ *   cu_seqlens   [B+1] int32 device array: prompt b is tokens cu_seqlens[b] .. cu_seqlens[b+1]-1
+ *                of the packed inputs; cu_seqlens[0] = 0, cu_seqlens[B] = total_tokens
+ *   total_tokens T, the packed token count
+ *   max_seq_len  host-side upper bound of the prompt lengths
+ *   q_c [T, n_h, d_h], q_r [T, n_h, d_r] (before RoPE), c_kv [T, d_c], k_r [T, d_r] (before
+ *                RoPE): bf16, row-major; q_c, c_kv 16-byte aligned
+ *   w_uk, w_uv   [n_h*d_h, d_c] bf16, 16-byte aligned (written before the call)
+ *   workspace    device scratch of workspace_bytes >= mla_prefill_workspace_size(dims, T),
+ *                256-byte aligned; its content on entry does not matter
+ *   o            [T, n_h, d_h] bf16, 16-byte aligned, written
+ *   lse          [T, n_h] fp32 natural-log normaliser, written (may be NULL)
+ * Errors: MLA_ERR_INVALID_ARG for bad sizes, null or misaligned pointers; a prompt table that
+ * is not as stated (or a prompt longer than max_seq_len) is reported by the device as
+ * MLA_ERR_BAD_SEQ_LEN through mla_get_last_device_error, with no access outside the buffers.
+ * ---------------------------------------------------------------------------------------- */
+size_t mla_prefill_workspace_size(const mla_dims_t *dims, int total_tokens);
+mla_status_t mla_prefill(const mla_dims_t *dims, int B, const int32_t *cu_seqlens, int total_tokens,
+                         int max_seq_len, const void *q_c, const void *q_r, const void *c_kv,
+                         const void *k_r, const void *w_uk, const void *w_uv, void *workspace,
+                         size_t workspace_bytes, void *o, float *lse, mla_stream_t stream);
+
+/* ----------------------------------------------------------------------------------------
  * Sequence split across GPUs (long contexts): exact merge of decode results.
  *
  * MLA article, section 한계 (limitations): every head reads the whole latent cache, so tensor

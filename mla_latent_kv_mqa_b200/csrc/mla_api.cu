@@ -247,6 +247,35 @@ mla_status_t mla_decode_fixed_scratch(const mla_dims_t *dims, int B, int s_q, co
                       kDecodeScratchBytes, o_lat, lse, stream);
 }
 
+size_t mla_prefill_workspace_size(const mla_dims_t *dims, int total_tokens) {
+    if (check_dims(dims) != MLA_OK || !prefill_supported(*dims) || total_tokens < 0) return 0;
+    return prefill_workspace_bytes(*dims, total_tokens);
+}
+
+mla_status_t mla_prefill(const mla_dims_t *dims, int B, const int32_t *cu_seqlens, int total_tokens,
+                         int max_seq_len, const void *q_c, const void *q_r, const void *c_kv,
+                         const void *k_r, const void *w_uk, const void *w_uv, void *workspace,
+                         size_t workspace_bytes, void *o, float *lse, mla_stream_t stream) {
+    mla_status_t s = check_dims(dims);
+    if (s != MLA_OK) return s;
+    if (!prefill_supported(*dims)) return MLA_ERR_UNSUPPORTED;
+    if (B < 0 || total_tokens < 0 || max_seq_len < 1) return MLA_ERR_INVALID_ARG;
+    if (B == 0 || total_tokens == 0) return MLA_OK;
+    // grid limits (heads, prompts, 128-token tiles) and int TMA coordinates over n_h * T rows
+    const int64_t T_pad = ((int64_t)total_tokens + 127) / 128 * 128;
+    if (B > 65535 || (int64_t)dims->n_h > 65535 || T_pad / 128 > 65535 ||
+        (int64_t)dims->n_h * T_pad > INT_MAX)
+        return MLA_ERR_INVALID_ARG;
+    if (!cu_seqlens || !q_c || !q_r || !c_kv || !k_r || !w_uk || !w_uv || !workspace || !o)
+        return MLA_ERR_INVALID_ARG;
+    if (!aligned(q_c, 16) || !aligned(c_kv, 16) || !aligned(w_uk, 16) || !aligned(w_uv, 16) || !aligned(o, 16) ||
+        !aligned(workspace, 256))
+        return MLA_ERR_INVALID_ARG;
+    if (workspace_bytes < prefill_workspace_bytes(*dims, total_tokens)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+    return from_cuda(launch_prefill(*dims, B, cu_seqlens, total_tokens, max_seq_len, q_c, q_r, c_kv, k_r, w_uk, w_uv,
+                                    workspace, workspace_bytes, o, lse, (cudaStream_t)stream));
+}
+
 mla_status_t mla_lse_merge_prepare(int rows, int n_h, int d_c, const float *o_lat, const float *lse,
                                    const float *lse_max, float *acc, mla_stream_t stream) {
     if (rows < 0 || n_h < 1 || d_c < 1 || (int64_t)rows * n_h > INT_MAX) return MLA_ERR_INVALID_ARG;

@@ -133,6 +133,13 @@ cudaError_t launch_combine_out_proj_tc(const mla_dims_t &d, int T, const int32_t
                                        float *o_lat, float *lse, const void *w_uv, void *o,
                                        mla_dtype_t out_dtype, cudaStream_t st);
 
+// MHA-mode prefill (d_h = 128, d_c = 512, d_R = 64, bf16, even n_h): K / V reconstruction
+// GEMM + causal tcgen05 attention over packed prompts (cu_seqlens [B + 1], T tokens).
+bool prefill_supported(const mla_dims_t &d);
+size_t prefill_workspace_bytes(const mla_dims_t &d, int T);
+cudaError_t launch_prefill(const mla_dims_t &d, int B, const int32_t *cu_seqlens, int T, int max_seq_len,
+                           const void *q_c, const void *q_r, const void *c_kv, const void *k_r, const void *w_uk,
+                           const void *w_uv, void *ws, size_t ws_bytes, void *o, float *lse, cudaStream_t st);
 // Sequence split across GPUs: the per-rank steps of the exact log-sum-exp merge.
 cudaError_t launch_lse_merge_prepare(int rows, int n_h, int d_c, const float *o_lat, const float *lse,
                                      const float *lse_max, float *acc, cudaStream_t st);

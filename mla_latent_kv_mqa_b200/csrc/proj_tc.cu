@@ -177,20 +177,23 @@ out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int n_h, con
 // multiply-adds), so o_lat and lse come out bit-identical to it:
 //     M = max_s m_s,  w_s = 2^(m_s - M),  L = sum_s w_s l_s,
 //     o_lat = sum_s w_s O_s / L,  lse = (M + log2 L) ln 2.
-// Grid (n_h, tiles of TNO rows) in clusters of 8 CTAs along the heads.  CTA q of the cluster
-// that owns heads 8g..8g+7 merges column block q (64 latent columns) for all 8 heads and all
-// rows of its tile: a warp's loads then read 8 heads x 4 bytes = one whole 32-byte sector per
-// column pair, where a CTA merging only its own head would use 4 bytes of every sector it
-// reads.  The merged values go, split into bf16 hi + lo exactly as out_proj splits o_lat,
+// Grid (n_h, tiles of TNO rows) in clusters of 4 CTAs along the heads (clusters of 8 would
+// not all fit on the GPU at once with one CTA per SM).  CTA q of the cluster that owns heads
+// 4g..4g+3 merges latent columns [128 q, 128 q + 128) for all 4 heads and all rows of its
+// tile: a warp's loads then read 4 heads x 4 bytes = half a 32-byte sector per column pair,
+// where a CTA merging only its own head would use 4 bytes of every sector it reads.  The merged values go, split into bf16 hi + lo exactly as out_proj splits o_lat,
 // straight into the B tile of the CTA that owns the head (st.async into a peer's shared
 // memory, completing on its b_full barrier; a plain store for the CTA's own head); o_lat and
 // lse are also written out.  Then every CTA runs
 // the out_proj MMAs of its head as out_proj_tc_kernel does.
 // ------------------------------------------------------------------------------------------
-constexpr int CO_CLUSTER = 8;
+constexpr int CO_CLUSTER = 4;
+constexpr int CO_COLS = DCL / CO_CLUSTER;   // latent columns merged per CTA: 128 = 2 column blocks
+constexpr int CO_THREADS = 256;
+constexpr int CO_FAST = 8;  // rows split over at most this many slots take the all-loads-first path
 
 template <typename To>
-__global__ void __cluster_dims__(CO_CLUSTER, 1, 1) __launch_bounds__(128, 1)
+__global__ void __cluster_dims__(CO_CLUSTER, 1, 1) __launch_bounds__(CO_THREADS, 1)
 combine_out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int n_h,
                            const int32_t *__restrict__ seg_range, const uint32_t *__restrict__ o_part,
                            const float *__restrict__ m_part, const float *__restrict__ l_part,
@@ -205,7 +208,7 @@ combine_out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int 
     const int h = blockIdx.x, t0 = blockIdx.y * TNO;
     const int nt = min(TNO, T - t0);
     const int npad = (nt + 15) & ~15;
-    const uint32_t q = cluster_ctarank();  // column block merged here; == h % 8
+    const uint32_t q = cluster_ctarank();  // merges latent columns [128 q, 128 q + 128); == h % 4
     const int hg = h - (int)q;             // first head of the cluster
 
     if (tid == 0) {
@@ -213,8 +216,9 @@ combine_out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int 
         mbar_init(smem_u32(&ctrl->b_full), 1);
         mbar_init(smem_u32(&ctrl->d_full), 1);
         ctrl->abort = 0;
-        // the 7 column blocks merged by the other CTAs of the cluster: nt rows x (hi + lo) x 128 B
-        mbar_arrive_expect_tx(smem_u32(&ctrl->b_full), (uint32_t)((CO_CLUSTER - 1) * nt * 256));
+        // the column blocks merged by the other CTAs of the cluster: 2 blocks per CTA, nt rows,
+        // hi + lo, 128 B each
+        mbar_arrive_expect_tx(smem_u32(&ctrl->b_full), (uint32_t)((CO_CLUSTER - 1) * nt * 512));
         fence_mbarrier_init_cluster();
         prefetch_tensormap(&tm_w);
         for (int kb = 0; kb < NWB; ++kb) {
@@ -232,40 +236,84 @@ combine_out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int 
     pdl_wait();      // the partials and the slot ranges are the decode's output
     const uint32_t bs = data_s + OP_B;
 
-    // ---- merge: thread = (head i of the cluster, 8-column chunk c of block q, row parity) ----
+    // ---- merge: thread = (head i of the cluster, 8-column chunk c of this CTA's 128, row r = rq mod 4) ----
+    // Every load a row needs is requested before any is used (up to CO_FAST slots), and the
+    // next row's slot range is requested before this row is merged, so a row costs about one
+    // round trip to L2.
     {
-        const int i = tid & 7, c = (tid >> 3) & 7;
+        const int i = tid & 3, c = (tid >> 2) & 15, rq = tid >> 6;
         const int hh = hg + i;
         const size_t slot_words = (size_t)(DCL / 2) * n_h;
-        const uint32_t *src = o_part + (size_t)(q * 32 + c * 4) * n_h + hh;
+        const uint32_t *src = o_part + (size_t)(q * (CO_COLS / 2) + c * 4) * n_h + hh;
         const uint32_t dst_bar = mapa(smem_u32(&ctrl->b_full), (uint32_t)i);
-        for (int r = tid >> 6; r < nt; r += 2) {
+        int s0 = 0, s1 = 0;
+        if (rq < nt) {
+            s0 = __ldcg(seg_range + 2 * (t0 + rq));
+            s1 = __ldcg(seg_range + 2 * (t0 + rq) + 1);
+        }
+        for (int r = rq; r < nt; r += CO_THREADS / 64) {
             const int row = t0 + r;
-            const int s0 = __ldcg(seg_range + 2 * row), s1 = __ldcg(seg_range + 2 * row + 1);
+            int n0 = 0, n1 = 0;
+            if (r + CO_THREADS / 64 < nt) {
+                n0 = __ldcg(seg_range + 2 * (row + CO_THREADS / 64));
+                n1 = __ldcg(seg_range + 2 * (row + CO_THREADS / 64) + 1);
+            }
             float M = -INFINITY, L = 0.f, acc[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-            for (int s = s0; s < s1; ++s) M = fmaxf(M, __ldcg(m_part + (size_t)s * n_h + hh));
-            for (int s = s0; s < s1; ++s) {
-                const float ms = __ldcg(m_part + (size_t)s * n_h + hh);
-                if (ms == -INFINITY) continue;  // empty slot: weight 0, partials never written
-                const float w = exp2f(ms - M);
-                L = fmaf(w, __ldcg(l_part + (size_t)s * n_h + hh), L);
-                uint32_t v[4];
+            if (s1 - s0 <= CO_FAST) {
+                float ms[CO_FAST], ls[CO_FAST];
+                uint32_t v[CO_FAST][4];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) v[k] = __ldcg(src + (size_t)s * slot_words + (size_t)k * n_h);
+                for (int j = 0; j < CO_FAST; ++j) {
+                    const int s = s0 + j;
+                    ms[j] = -INFINITY;
+                    ls[j] = 0.f;
+                    if (s < s1) {
+                        ms[j] = __ldcg(m_part + (size_t)s * n_h + hh);
+                        ls[j] = __ldcg(l_part + (size_t)s * n_h + hh);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    acc[2 * k] = fmaf(w, __uint_as_float(v[k] << 16), acc[2 * k]);
-                    acc[2 * k + 1] = fmaf(w, __uint_as_float(v[k] & 0xffff0000u), acc[2 * k + 1]);
+                        for (int k = 0; k < 4; ++k) v[j][k] = __ldcg(src + (size_t)s * slot_words + (size_t)k * n_h);
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < CO_FAST; ++j) M = fmaxf(M, ms[j]);
+#pragma unroll
+                for (int j = 0; j < CO_FAST; ++j) {
+                    if (ms[j] == -INFINITY) continue;  // empty or past the range: weight 0, never read
+                    const float w = exp2f(ms[j] - M);
+                    L = fmaf(w, ls[j], L);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        acc[2 * k] = fmaf(w, __uint_as_float(v[j][k] << 16), acc[2 * k]);
+                        acc[2 * k + 1] = fmaf(w, __uint_as_float(v[j][k] & 0xffff0000u), acc[2 * k + 1]);
+                    }
+                }
+            } else {
+                for (int s = s0; s < s1; ++s) M = fmaxf(M, __ldcg(m_part + (size_t)s * n_h + hh));
+                for (int s = s0; s < s1; ++s) {
+                    const float ms = __ldcg(m_part + (size_t)s * n_h + hh);
+                    if (ms == -INFINITY) continue;
+                    const float w = exp2f(ms - M);
+                    L = fmaf(w, __ldcg(l_part + (size_t)s * n_h + hh), L);
+                    uint32_t v[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) v[k] = __ldcg(src + (size_t)s * slot_words + (size_t)k * n_h);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        acc[2 * k] = fmaf(w, __uint_as_float(v[k] << 16), acc[2 * k]);
+                        acc[2 * k + 1] = fmaf(w, __uint_as_float(v[k] & 0xffff0000u), acc[2 * k + 1]);
+                    }
                 }
             }
+            s0 = n0;
+            s1 = n1;
             const float inv = L > 0.f ? 1.f / L : 0.f;
             float x[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) x[j] = acc[j] * inv;
             if (o_lat) {
-                float4 *dst = reinterpret_cast<float4 *>(o_lat + ((size_t)row * n_h + hh) * DCL + q * 64 + c * 8);
+                float4 *dst = reinterpret_cast<float4 *>(o_lat + ((size_t)row * n_h + hh) * DCL + q * CO_COLS + c * 8);
                 dst[0] = make_float4(x[0], x[1], x[2], x[3]);
                 dst[1] = make_float4(x[4], x[5], x[6], x[7]);
             }
@@ -280,7 +328,7 @@ combine_out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int 
                 hw[k] = *reinterpret_cast<const uint32_t *>(&hv);
                 lw[k] = *reinterpret_cast<const uint32_t *>(&lv);
             }
-            const uint32_t loc = bs + q * OP_BBLK + r * 128 + ((c ^ (r & 7)) << 4);
+            const uint32_t loc = bs + (2 * q + (c >> 3)) * OP_BBLK + r * 128 + (((c & 7) ^ (r & 7)) << 4);
             if (i == (int)q) {  // this CTA's own head: a plain shared-memory store
                 st_shared_v4(loc, hw[0], hw[1], hw[2], hw[3]);
                 st_shared_v4(loc + TNO * 128, lw[0], lw[1], lw[2], lw[3]);
@@ -292,7 +340,7 @@ combine_out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int 
         }
     }
     // rows nt..npad-1 of the MMA's N are zero (only rows < nt are merged)
-    for (int idx = tid; idx < (npad - nt) * 64; idx += 128) {
+    for (int idx = tid; idx < (npad - nt) * 64; idx += CO_THREADS) {
         const int r = nt + (idx >> 6), g = idx & 63, c = g & 7;
         const uint32_t hs = bs + (g >> 3) * OP_BBLK + r * 128 + ((c ^ (r & 7)) << 4);
         st_shared_v4(hs, 0u, 0u, 0u, 0u);
@@ -327,14 +375,16 @@ combine_out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int 
     bool ok = __syncthreads_and(*abort_flag == 0);
     if (ok) ok = __syncthreads_and(wait(smem_u32(&ctrl->d_full), 0, abort_flag));
     if (ok) {
-        tc_fence_after();
-        const int d = warp * 32 + lane;
-        uint32_t v[32];
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16), v);
-        tmem_wait_ld();
+        if (warp < 4) {  // the accumulator's 128 lanes = the head's 128 output rows
+            tc_fence_after();
+            const int d = warp * 32 + lane;
+            uint32_t v[32];
+            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16), v);
+            tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-            if (j < nt) o[((size_t)(t0 + j) * n_h + h) * DH + d] = from_f32<To>(__uint_as_float(v[j]));
+            for (int j = 0; j < 32; ++j)
+                if (j < nt) o[((size_t)(t0 + j) * n_h + h) * DH + d] = from_f32<To>(__uint_as_float(v[j]));
+        }
     } else if (tid == 0) {
         record_error(err, kErrTimeout);
     }
@@ -504,7 +554,8 @@ namespace {
 // stream: their blocks start (and fetch the constant weights) while that kernel drains, and wait
 // for it on the device before they read an activation or write an output.
 template <typename... Exp, typename... Act>
-cudaError_t launch_dependent(void (*kernel)(Exp...), dim3 grid, int smem, cudaStream_t st, Act &&...args) {
+cudaError_t launch_dependent_n(void (*kernel)(Exp...), dim3 grid, int threads, int smem, cudaStream_t st,
+                               Act &&...args) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchAttribute pdl;
@@ -512,7 +563,7 @@ cudaError_t launch_dependent(void (*kernel)(Exp...), dim3 grid, int smem, cudaSt
     pdl.val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
-    cfg.blockDim = dim3(128);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cfg.attrs = &pdl;
@@ -522,6 +573,10 @@ cudaError_t launch_dependent(void (*kernel)(Exp...), dim3 grid, int smem, cudaSt
     cfg.numAttrs = 1;
 #endif
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<Act &&>(args)...);
+}
+template <typename... Exp, typename... Act>
+cudaError_t launch_dependent(void (*kernel)(Exp...), dim3 grid, int smem, cudaStream_t st, Act &&...args) {
+    return launch_dependent_n(kernel, grid, 128, smem, st, static_cast<Act &&>(args)...);
 }
 }  // namespace
 
@@ -556,12 +611,12 @@ cudaError_t launch_combine_out_proj_tc(const mla_dims_t &d, int T, const int32_t
     if (!tmap_bf16_2d(&tm, w_uv, DCL, (uint64_t)d.n_h * DH, DCL * 2, 64, 128)) return cudaErrorInvalidValue;
     const dim3 grid(d.n_h, (T + TNO - 1) / TNO);
     if (out_dtype == MLA_DTYPE_BF16)
-        return launch_dependent(combine_out_proj_tc_kernel<__nv_bfloat16>, grid, OP_SMEM, st, tm, T, d.n_h,
-                                seg_range, o_part, m_part, l_part, o_lat, lse,
-                                reinterpret_cast<__nv_bfloat16 *>(o), device_error_word());
-    return launch_dependent(combine_out_proj_tc_kernel<float>, grid, OP_SMEM, st, tm, T, d.n_h, seg_range,
-                            o_part, m_part, l_part, o_lat, lse, reinterpret_cast<float *>(o),
-                            device_error_word());
+        return launch_dependent_n(combine_out_proj_tc_kernel<__nv_bfloat16>, grid, CO_THREADS, OP_SMEM, st, tm, T,
+                                  d.n_h, seg_range, o_part, m_part, l_part, o_lat, lse,
+                                  reinterpret_cast<__nv_bfloat16 *>(o), device_error_word());
+    return launch_dependent_n(combine_out_proj_tc_kernel<float>, grid, CO_THREADS, OP_SMEM, st, tm, T, d.n_h,
+                              seg_range, o_part, m_part, l_part, o_lat, lse, reinterpret_cast<float *>(o),
+                              device_error_word());
 }
 
 }  // namespace mla

@@ -62,8 +62,8 @@ class PagedLatentCache:
 
 
 class MLADecodeLayer:
-    """Weights of one absorbed-MLA layer (W_UK, W_UV as [n_h*d_h, d_c]) plus a reusable
-    decode workspace."""
+    """Weights of one MLA layer (W_UK, W_UV as [n_h*d_h, d_c]) plus reusable decode and
+    prefill workspaces."""
 
     def __init__(self, dims: N.mla_dims_t, w_uk: torch.Tensor, w_uv: torch.Tensor):
         self.dims = dims
@@ -72,6 +72,7 @@ class MLADecodeLayer:
         self.device = w_uk.device
         self._ws = None
         self._ws_key = None
+        self._pf_ws = None
 
     # -- the four calls ----------------------------------------------------------------------
     def append(self, cache: PagedLatentCache, c_kv, k_r, seq_idx, pos, block_table, stream=None):
@@ -130,6 +131,23 @@ class MLADecodeLayer:
                              max_blocks, cache.num_blocks, seq_lens, max_seq_len, ws, ws.numel(), self.w_uv,
                              o, dt, o_lat, lse, stream)
         return o, o_lat, lse
+
+    def prefill(self, q_c, q_r, c_kv, k_r, cu_seqlens, max_seq_len, o=None, lse=None, stream=None):
+        """Causal MHA-mode attention over packed prompts (cu_seqlens [B + 1] int32 on the
+        device); returns (o [T, n_h, d_h] bf16, lse [T, n_h])."""
+        d = self.dims
+        T = q_c.shape[0]
+        B = cu_seqlens.numel() - 1
+        if o is None:
+            o = torch.empty((T, d.n_h, d.d_h), dtype=torch.bfloat16, device=self.device)
+        if lse is None:
+            lse = torch.empty((T, d.n_h), dtype=torch.float32, device=self.device)
+        n = N.mla_prefill_workspace_size(d, T)
+        if self._pf_ws is None or self._pf_ws.numel() < n:
+            self._pf_ws = torch.empty(max(n, 256), dtype=torch.uint8, device=self.device)
+        N.mla_prefill(d, B, cu_seqlens, T, max_seq_len, q_c, q_r, c_kv, k_r, self.w_uk, self.w_uv, self._pf_ws,
+                      self._pf_ws.numel(), o, lse, stream)
+        return o, lse
 
     def out_proj(self, o_lat, out_dtype="f32", out=None, stream=None):
         d = self.dims

@@ -70,6 +70,9 @@ _lib.mla_decode_fixed_scratch.argtypes = [_dp, _i, _i, _vp, _vp, _vp, _vp, _vp, 
 _lib.mla_out_proj.argtypes = [_dp, _i, _vp, _vp, _vp, _i, _vp]
 _lib.mla_decode_project.argtypes = [_dp, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _i, _vp, _sz,
                                     _vp, _vp, _i, _vp, _vp, _vp]
+_lib.mla_prefill_workspace_size.argtypes = [_dp, _i]
+_lib.mla_prefill_workspace_size.restype = _sz
+_lib.mla_prefill.argtypes = [_dp, _i, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp]
 _lib.mla_lse_merge_prepare.argtypes = [_i, _i, _i, _vp, _vp, _vp, _vp, _vp]
 _lib.mla_lse_merge_finish.argtypes = [_i, _i, _i, _vp, _vp, _vp, _vp, _vp]
 _lib.mla_get_last_device_error.argtypes = []
@@ -77,7 +80,7 @@ _lib.mla_status_string.argtypes = [_i]
 _lib.mla_status_string.restype = ctypes.c_char_p
 _lib.mla_version.restype = _i
 for _f in ("mla_absorb_q", "mla_cache_append", "mla_decode", "mla_decode_fixed_scratch", "mla_out_proj",
-           "mla_decode_project", "mla_get_last_device_error", "mla_lse_merge_prepare",
+           "mla_decode_project", "mla_prefill", "mla_get_last_device_error", "mla_lse_merge_prepare",
            "mla_lse_merge_finish"):
     getattr(_lib, _f).restype = _i
 
@@ -174,6 +177,17 @@ def mla_decode_project(dims, B, s_q, q_abs, kv_pool, kr_pool, kv_scale, block_ta
                                    _ptr(seq_lens), max_seq_len, _ptr(workspace), workspace_bytes, _ptr(w_uv),
                                    _ptr(o), out_dtype, _ptr(o_lat), _ptr(lse), _stream(stream)),
            "mla_decode_project")
+
+
+def mla_prefill_workspace_size(dims, total_tokens) -> int:
+    return int(_lib.mla_prefill_workspace_size(ctypes.byref(dims), total_tokens))
+
+
+def mla_prefill(dims, B, cu_seqlens, total_tokens, max_seq_len, q_c, q_r, c_kv, k_r, w_uk, w_uv, workspace,
+                workspace_bytes, o, lse=None, stream=None):
+    _check(_lib.mla_prefill(ctypes.byref(dims), B, _ptr(cu_seqlens), total_tokens, max_seq_len, _ptr(q_c), _ptr(q_r),
+                            _ptr(c_kv), _ptr(k_r), _ptr(w_uk), _ptr(w_uv), _ptr(workspace), workspace_bytes, _ptr(o),
+                            _ptr(lse), _stream(stream)), "mla_prefill")
 
 
 def mla_lse_merge_prepare(rows, n_h, d_c, o_lat, lse, lse_max, acc, stream=None):

@@ -223,6 +223,50 @@ def make_decode(seed: int, seq_lens, *, s_q: int = 1, kv_dtype: str = "bf16",
     return wl
 
 
+@dataclass
+class PrefillWorkload:
+    """Causal prefill of B prompts packed into T tokens (prompt b is tokens cu_seqlens[b] ..
+    cu_seqlens[b+1]-1, token i of a prompt at position i).  Arrays as in DecodeWorkload:
+    float32 holding bf16 values; q_r and k_r before RoPE."""
+    name: str
+    dims: MLADims
+    seq_lens: np.ndarray              # [B] int32
+    cu_seqlens: np.ndarray            # [B+1] int32
+    q_c: np.ndarray                   # [T, n_h, d_h]
+    q_r: np.ndarray                   # [T, n_h, d_r]
+    c_kv: np.ndarray                  # [T, d_c]
+    k_r: np.ndarray                   # [T, d_r]
+    w_uk: np.ndarray                  # [n_h*d_h, d_c]
+    w_uv: np.ndarray                  # [n_h*d_h, d_c]
+
+    @property
+    def B(self) -> int:
+        return int(self.seq_lens.shape[0])
+
+    @property
+    def T(self) -> int:
+        return int(self.cu_seqlens[-1])
+
+
+def make_prefill(seed: int, seq_lens, dims: MLADims = V3_DIMS, name: str = "prefill") -> PrefillWorkload:
+    """Prompts of the given lengths, V3-shaped by default: weights ~ N(0, 1/d_c), activations
+    and latents ~ N(0, 1), all rounded to bf16 (the decode workloads' recipe)."""
+    rng = np.random.default_rng(seed)
+    seq_lens = np.asarray(seq_lens, dtype=np.int32)
+    cu = np.zeros(len(seq_lens) + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(seq_lens)
+    T = int(cu[-1])
+    w_std = 1.0 / np.sqrt(dims.d_c)
+    w_uk = _normal(rng, (dims.n_h * dims.d_h, dims.d_c), w_std)
+    w_uv = _normal(rng, (dims.n_h * dims.d_h, dims.d_c), w_std)
+    q_c = _normal(rng, (T, dims.n_h, dims.d_h))
+    q_r = _normal(rng, (T, dims.n_h, dims.d_r))
+    c_kv = _normal(rng, (T, dims.d_c))
+    k_r = _normal(rng, (T, dims.d_r))
+    return PrefillWorkload(name=name, dims=dims, seq_lens=seq_lens, cu_seqlens=cu, q_c=q_c, q_r=q_r,
+                           c_kv=c_kv, k_r=k_r, w_uk=w_uk, w_uv=w_uv)
+
+
 CONFIGS = {
     "toy": dict(desc="Toy MLA layer d=1024 n_h=8 d_h=64 d_c=128 d_cq=256 d_R=32, B=1, ctx 256, fp32"),
     "v3": dict(desc="DeepSeek-V3-shaped decode n_h=128 d_h=128 d_c=512 d_R=64, bf16, B=16, ctx 4096, page 64"),

@@ -20,9 +20,11 @@ def max_abs(x, ref) -> float:
 
 # Tolerances of the bf16 path: relative L2 <= 4e-3 and max |err| <= 2e-2 on o_lat and o, and
 # |err(lse)| <= 1e-2.  Workloads whose per-token norms are log-normal (the long-context recipe)
-# use max |err| <= 2e-2 * max(1, max |ref|) and |err(lse)| <= 1e-2 * max(1, |lse|) instead:
-# tests/test_tolerance_reading.py shows that exact arithmetic on the bf16 operands the C ABI
-# defines already exceeds the flat bounds there, and stays far inside them on N(0,1) latents.
+# use max |err| <= 2e-2 * max(1, max |ref|) and |err(lse)| <= 1e-2 * max(1, |lse|) instead, and
+# hold the relative L2 bound against the oracle run on the bf16 operands the C ABI defines
+# (rounded_operand_ref): tests/test_tolerance_reading.py shows that exact arithmetic on those
+# operands already exceeds the flat bounds there -- and on some seeds the relative L2 bound as
+# well -- while it stays far inside all of them on N(0,1) latents.
 # FP8 content cache: relative L2 <= 3e-2 against the oracle on its own dequantised cache.
 BF16_REL, BF16_ABS, FP8_REL, LSE_ABS = 4e-3, 2e-2, 3e-2, 1e-2
 
@@ -34,12 +36,14 @@ def scaled_max_abs(x, ref):
     return float(np.abs(x - ref).max() / max(1.0, float(np.abs(ref).max())))
 
 
-def check_step(got, ref, rows, heads, rel_tol, abs_tol, *, lognormal=False):
+def check_step(got, ref, rows, heads, rel_tol, abs_tol, *, lognormal=False, ref_ops=None):
     """Compare one step's (o_lat, lse, o) on the given rows and heads with the oracle's.
 
     ``lognormal``: the workload's per-token norms are log-normal; the max-abs and lse bounds
-    scale with the output (see the tolerance note above).  Both the plain and the scaled
-    errors are always reported in the assertion message."""
+    scale with the output (see the tolerance note above).  ``ref_ops``: the oracle on the
+    boundary's bf16 operands (rounded_operand_ref); when given, the relative L2 bound applies
+    against it (the kernel's own error) and is also reported against ``ref``.  Both the plain
+    and the scaled errors are always reported in the assertion message."""
     q_abs, o_lat, lse, o = got
     o_lat = o_lat.cpu().numpy()[rows][:, heads]
     o = o.float().cpu().numpy()[rows][:, heads]
@@ -50,12 +54,79 @@ def check_step(got, ref, rows, heads, rel_tol, abs_tol, *, lognormal=False):
              o_lat_scaled=scaled_max_abs(o_lat, ref.o_lat), o_scaled=scaled_max_abs(o, ref.o),
              lse_abs=float(dl.max()), lse_scaled=float(np.max(dl / np.maximum(1.0, np.abs(ref.lse)))),
              bounds="scaled (log-normal norms)" if lognormal else "flat")
-    assert e["o_lat_rel"] <= rel_tol and e["o_rel"] <= rel_tol, e
+    rel = (e["o_lat_rel"], e["o_rel"])
+    if ref_ops is not None:
+        e["o_lat_rel_vs_operands"] = rel_l2(o_lat, ref_ops.o_lat)
+        e["o_rel_vs_operands"] = rel_l2(o, ref_ops.o)
+        rel = (e["o_lat_rel_vs_operands"], e["o_rel_vs_operands"])
+    assert rel[0] <= rel_tol and rel[1] <= rel_tol, e
     k = "_scaled" if lognormal else "_abs"
     if abs_tol is not None:
         assert e["o_lat" + k] <= abs_tol and e["o" + k] <= abs_tol, e
     assert e["lse" + k] <= LSE_ABS, e
     return e
+
+
+def bf16_round(x):
+    """Round to bf16 (nearest even) and return float64."""
+    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.bfloat16).double().numpy()
+
+
+def rope_rows(x, pos, base=1e4):
+    """Half-split rotation of the rows of x [n, d] by angles pos[n] * base^(-2k/d) (the MLA
+    article's implementation-section pairing), vectorised; used only to prepare rounded
+    oracle inputs."""
+    d = x.shape[1]
+    half = d // 2
+    ang = np.asarray(pos, dtype=np.float64)[:, None] * base ** (-2.0 * np.arange(half) / d)[None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = x[:, :half], x[:, half:]
+    return np.concatenate([a * c - b * s, b * c + a * s], 1)
+
+
+def rounded_operand_ref(wl: W.DecodeWorkload, orc, seqs, heads):
+    """The fp64 oracle on the operands the C ABI fixes for the bf16 path: the absorbed query
+    q_lat and the rotated RoPE query rounded to bf16 (what mla_absorb_q writes), the rotated
+    RoPE key rounded to bf16 (what mla_cache_append stores); every other step exact.  s_q = 1:
+    q_lat is rounded by a rank-one update of each head's W^UK (one query row per head), the
+    rotations by handing the oracle RoPE(bf16(RoPE(x, p)), -p).  Returns (rows, heads, result)
+    like oracle_ref."""
+    from oracle.oracle import DecodeResult
+    assert wl.s_q == 1 and wl.kv_dtype == "bf16"
+    d = wl.dims
+    heads = np.asarray(heads)
+    wsel = (heads[:, None] * d.d_h + np.arange(d.d_h)[None, :]).reshape(-1)
+    wuk = wl.w_uk[wsel].astype(np.float64)
+    wuv = wl.w_uv[wsel].astype(np.float64)
+    outs = []
+    for b in seqs:
+        qc = wl.q_c[[b]][:, heads].astype(np.float64)
+        qr = wl.q_r[[b]][:, heads].astype(np.float64)
+        c = wl.seq_c_kv(b).astype(np.float64)
+        k = wl.seq_k_r(b).astype(np.float64)
+        qp = wl.q_pos[[b]]
+        exact = orc.decode_absorbed(qc, qr, qp, [c], [k], wuk, wuv, rope_base=d.rope_base)
+        tgt = bf16_round(exact.q_lat)
+        w2 = wuk.reshape(len(heads), d.d_h, d.d_c).copy()
+        for i in range(len(heads)):
+            q = qc[0, i]
+            w2[i] += np.outer(q, tgt[0, i] - exact.q_lat[0, i]) / (q @ q)
+        pq = np.full(len(heads), int(qp[0]))
+        qr2 = rope_rows(bf16_round(rope_rows(qr[0], pq, d.rope_base)), -pq, d.rope_base)[None]
+        j = np.arange(c.shape[0])
+        k2 = rope_rows(bf16_round(rope_rows(k, j, d.rope_base)), -j, d.rope_base)
+        outs.append(orc.decode_absorbed(qc, qr2, qp, [c], [k2], w2.reshape(-1, d.d_c), wuv, rope_base=d.rope_base))
+    res = DecodeResult(o=np.concatenate([r.o for r in outs]), lse=np.concatenate([r.lse for r in outs]),
+                       o_lat=np.concatenate([r.o_lat for r in outs]))
+    return np.asarray(list(seqs)), heads, res
+
+
+def operands_ref(wl: W.DecodeWorkload, orc, rows, heads):
+    """rounded_operand_ref where the relative bound is applied against it (bf16 cache, s_q = 1,
+    log-normal norms), else None."""
+    if wl.extra.get("lognormal_norms", False) and wl.kv_dtype == "bf16" and wl.s_q == 1:
+        return rounded_operand_ref(wl, orc, list(rows), heads)[2]
+    return None
 
 
 def _act(x: np.ndarray, act: str, dev):
@@ -127,3 +198,41 @@ def oracle_ref(wl: W.DecodeWorkload, orc, seqs=None, heads=None, naive=False):
     if naive:
         return rows, heads, orc.decode_naive(*args, s_q=wl.s_q, rope_base=d.rope_base)
     return rows, heads, orc.decode_absorbed(*args, s_q=wl.s_q, rope_base=d.rope_base)
+
+
+class PrefillRun:
+    """Device state of one prefill workload and the call through the C ABI."""
+
+    def __init__(self, wl: W.PrefillWorkload, dev="cuda"):
+        from mla_latent_kv_mqa_b200 import layer as Lyr
+        self.wl = wl
+        d = wl.dims
+        self.dims = Lyr.dims_for(d.n_h, d.d_h, d.d_c, d.d_r, act="bf16", kv="bf16", page=d.page,
+                                 rope_base=d.rope_base)
+        self.layer = Lyr.MLADecodeLayer(self.dims, _act(wl.w_uk, "bf16", dev), _act(wl.w_uv, "bf16", dev))
+        self.cu = torch.from_numpy(wl.cu_seqlens.astype(np.int32)).to(dev)
+        self.max_len = int(wl.seq_lens.max())
+        self.q_c = _act(wl.q_c, "bf16", dev)
+        self.q_r = _act(wl.q_r, "bf16", dev)
+        self.c_kv = _act(wl.c_kv, "bf16", dev)
+        self.k_r = _act(wl.k_r, "bf16", dev)
+
+    def run(self, o=None, lse=None):
+        o, lse = self.layer.prefill(self.q_c, self.q_r, self.c_kv, self.k_r, self.cu, self.max_len, o=o, lse=lse)
+        torch.cuda.synchronize()
+        return o, lse
+
+
+def prefill_oracle_rows(wl: W.PrefillWorkload, orc, rows, heads):
+    """Naive-mode (MHA) oracle for the given (prompt, token) rows and heads: each sampled row is
+    a one-query problem whose context is its prompt's tokens 0..t."""
+    d = wl.dims
+    heads = np.asarray(heads)
+    wsel = (heads[:, None] * d.d_h + np.arange(d.d_h)[None, :]).reshape(-1)
+    glob = np.array([wl.cu_seqlens[b] + t for b, t in rows])
+    cs = [np.asarray(wl.c_kv[wl.cu_seqlens[b]:wl.cu_seqlens[b] + t + 1], dtype=np.float64) for b, t in rows]
+    ks = [np.asarray(wl.k_r[wl.cu_seqlens[b]:wl.cu_seqlens[b] + t + 1], dtype=np.float64) for b, t in rows]
+    pos = np.array([t for _, t in rows], dtype=np.int64)
+    ref = orc.decode_naive(wl.q_c[glob][:, heads], wl.q_r[glob][:, heads], pos, cs, ks, wl.w_uk[wsel],
+                           wl.w_uv[wsel], s_q=1, rope_base=d.rope_base)
+    return glob, heads, ref

@@ -88,6 +88,21 @@ def test_host_argument_checks(N):
     assert dp_call(q_abs=None) == N.MLA_ERR_INVALID_ARG
     assert dp_call(out_dtype=N.MLA_DTYPE_FP8_E4M3) == N.MLA_ERR_UNSUPPORTED
     assert dp_call(B=0, w_uv=None) == N.MLA_OK
+    # prefill: the supported shape, sizes, null and misaligned pointers, workspace size
+    def pf(B=2, T=256, max_len=128, cu=16, q_c=16, o=16, ws=256, ws_bytes=1 << 40, d=dp):
+        return L.mla_prefill(d, B, cu, T, max_len, q_c, 16, 16, 16, 16, 16, ws, ws_bytes, o, None, None)
+    assert pf(B=0) == N.MLA_OK and pf(T=0) == N.MLA_OK
+    assert pf(B=-1) == N.MLA_ERR_INVALID_ARG and pf(max_len=0) == N.MLA_ERR_INVALID_ARG
+    assert pf(cu=None) == N.MLA_ERR_INVALID_ARG and pf(q_c=8) == N.MLA_ERR_INVALID_ARG
+    assert pf(o=8) == N.MLA_ERR_INVALID_ARG and pf(ws=16) == N.MLA_ERR_INVALID_ARG
+    assert pf(ws_bytes=1024) == N.MLA_ERR_WORKSPACE_TOO_SMALL
+    assert pf(B=70000) == N.MLA_ERR_INVALID_ARG
+    odd = _v3(N)
+    odd.n_h = 3
+    assert pf(d=ctypes.byref(odd)) == N.MLA_ERR_UNSUPPORTED
+    assert N.mla_prefill_workspace_size(odd, 256) == 0
+    w1, w2 = N.mla_prefill_workspace_size(d, 256), N.mla_prefill_workspace_size(d, 257)
+    assert 0 < w1 < w2
     # sequence-split merge: sizes, null pointers with work to do, (rows, n_h) within int
     for f in (L.mla_lse_merge_prepare, L.mla_lse_merge_finish):
         for rows, n_h, d_c in [(-1, 1, 1), (1, 0, 1), (1, 1, 0), (1 << 20, 1 << 12, 8)]:

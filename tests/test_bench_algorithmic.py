@@ -44,3 +44,19 @@ def test_varlen_lengths_and_bytes():
     b, f = bench.algorithmic(_wl(lens))
     assert b == int(lens.sum()) * 1152
     assert 0.55e9 < b < 0.75e9  # about 642 MB for U[1024, 16384] at B = 64
+
+
+def test_prefill_flops_count_every_visible_pair():
+    """Brute force over (query t, key j <= t) pairs of small prompts, and the benchmark's
+    4 x 4096 prompts: 2 (d_h + d_R) + 2 d_h FLOPs per head and pair, plus 2 d_c d_h per head,
+    token and reconstructed matrix (K and V)."""
+    d = W.V3_DIMS
+    lens = [1, 5, 130]
+    pairs = sum(1 for L in lens for t in range(L) for j in range(t + 1))
+    wl = types.SimpleNamespace(dims=d, seq_lens=np.asarray(lens, np.int32), T=sum(lens))
+    attn, up = bench.prefill_flops(wl)
+    assert attn == pairs * d.n_h * 2 * (192 + 128)
+    assert up == 2 * sum(lens) * 2 * 512 * 128 * 128
+    wl = types.SimpleNamespace(dims=d, seq_lens=np.asarray(bench.PREFILL_LENS, np.int32), T=4 * 4096)
+    attn, up = bench.prefill_flops(wl)
+    assert attn == 4 * (4096 * 4097 // 2) * 128 * 640 and up == 549_755_813_888

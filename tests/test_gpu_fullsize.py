@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from mla_latent_kv_mqa_b200 import workloads as W
-from tests.harness import BF16_ABS, BF16_REL, FP8_REL, GpuRun, check_step, oracle_ref
+from tests.harness import BF16_ABS, BF16_REL, FP8_REL, GpuRun, check_step, operands_ref, oracle_ref
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -46,4 +46,5 @@ def test_full_size_sampled_rows(oracle_mod, cfg):
     rows, heads, ref = oracle_ref(wl, oracle_mod, seqs, heads)
     fp8 = wl.kv_dtype == "fp8"
     check_step(got, ref, rows, heads, FP8_REL if fp8 else BF16_REL, None if fp8 else BF16_ABS,
-               lognormal=wl.extra.get("lognormal_norms", False))
+               lognormal=wl.extra.get("lognormal_norms", False),
+               ref_ops=operands_ref(wl, oracle_mod, rows, heads))

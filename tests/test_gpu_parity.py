@@ -13,8 +13,8 @@ import pytest
 import torch
 
 from mla_latent_kv_mqa_b200 import workloads as W
-from tests.harness import (BF16_ABS, BF16_REL, FP8_REL, LSE_ABS, GpuRun, check_step, max_abs, oracle_ref,
-                           rel_l2, scaled_max_abs)
+from tests.harness import (BF16_ABS, BF16_REL, FP8_REL, LSE_ABS, GpuRun, check_step, max_abs, operands_ref,
+                           oracle_ref, rel_l2, scaled_max_abs)
 
 pytestmark = pytest.mark.gpu
 
@@ -29,9 +29,10 @@ def _cuda():
     torch.backends.cuda.matmul.allow_tf32 = False
 
 
-def _check(wl, got, ref, rows, heads, rel_tol, abs_tol):
+def _check(wl, got, ref, rows, heads, rel_tol, abs_tol, orc=None):
     return check_step(got, ref, rows, heads, rel_tol, abs_tol,
-                      lognormal=wl.extra.get("lognormal_norms", False))
+                      lognormal=wl.extra.get("lognormal_norms", False),
+                      ref_ops=operands_ref(wl, orc, rows, heads) if orc is not None else None)
 
 
 # ---------------------------------------------------------------------------------------------
@@ -61,7 +62,7 @@ def test_decode_matches_oracle_small(oracle_mod, case, simt):
     got = run.step()
     rows, heads, ref = oracle_ref(wl, oracle_mod)
     tol = FP8_REL if wl.kv_dtype == "fp8" else BF16_REL
-    _check(wl, got, ref, rows, heads, tol, None if wl.kv_dtype == "fp8" else BF16_ABS)
+    _check(wl, got, ref, rows, heads, tol, None if wl.kv_dtype == "fp8" else BF16_ABS, oracle_mod)
     # q_abs = [W_UK^T q_C ; RoPE(q_R)] against the oracle's q_lat and rotation
     q_abs = got[0].float().cpu().numpy()
     assert rel_l2(q_abs[:, :, :wl.dims.d_c], ref.q_lat) <= 4e-3

@@ -18,7 +18,7 @@ import torch
 from mla_latent_kv_mqa_b200 import native as N
 from mla_latent_kv_mqa_b200 import seqsplit as S
 from mla_latent_kv_mqa_b200 import workloads as W
-from tests.harness import BF16_ABS, BF16_REL, FP8_REL, GpuRun, check_step, oracle_ref, rel_l2
+from tests.harness import BF16_ABS, BF16_REL, FP8_REL, GpuRun, check_step, operands_ref, oracle_ref, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -82,7 +82,8 @@ def test_split_decode_matches_the_oracle_on_whole_sequences(oracle_mod, case):
     rows, heads, ref = oracle_ref(wl, oracle_mod)
     fp8 = wl.kv_dtype == "fp8"
     check_step((q_abs, o_lat, lse, o), ref, rows, heads, FP8_REL if fp8 else BF16_REL,
-               None if fp8 else BF16_ABS, lognormal=wl.extra.get("lognormal_norms", False))
+               None if fp8 else BF16_ABS, lognormal=wl.extra.get("lognormal_norms", False),
+               ref_ops=operands_ref(wl, oracle_mod, rows, heads))
     # the split is real: one rank's partial alone is far from the answer
     assert rel_l2(parts[0][0].cpu().numpy(), ref.o_lat) > 0.05
     # and the merge agrees with the unsplit decode of the same cache

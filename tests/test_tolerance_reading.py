@@ -15,7 +15,9 @@ Findings pinned here, which decide how tests/harness.check_step applies the boun
   |o_lat| ~ 20 and lse ~ 9..22, and the rounding alone moves single elements of o_lat by more
   than 2e-2 and lse by more than 1e-2.  No kernel can meet the flat bounds there, so those
   cases (and only those) use max |err| <= 2e-2 * max(1, max |ref|) and
-  |err(lse)| <= 1e-2 * max(1, |lse|).  Relative L2 stays inside 4e-3 in every case.
+  |err(lse)| <= 1e-2 * max(1, |lse|).  The relative L2 of the rounding alone is 3.5e-3 on
+  seed 23 but 4.4e-3 on seed 64, above the 4e-3 bound: on these cases the relative bound
+  is held against the oracle on the rounded operands (the kernel's own error).
 
 The rounding is applied to the oracle's INPUTS only (oracle/ is unchanged):
 * q_lat: the oracle forms q_lat = W^UK_h^T q^C itself, so W^UK_h gets the rank-one update
@@ -26,26 +28,14 @@ The rounding is applied to the oracle's INPUTS only (oracle/ is unchanged):
 """
 import numpy as np
 import pytest
-import torch
 
 from mla_latent_kv_mqa_b200 import workloads as W
 
 FLAT_ABS, REL, LSE_ABS = 2e-2, 4e-3, 1e-2
 
 
-def _bf16(x):
-    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.bfloat16).double().numpy()
-
-
-def _rope_np(x, pos, base=1e4):
-    """Half-split rotation of the rows of x [n, d] by angles pos[n] * base^(-2k/d) (the
-    implementation section's pairing), vectorised; used only to prepare rounded inputs."""
-    d = x.shape[1]
-    half = d // 2
-    ang = np.asarray(pos, dtype=np.float64)[:, None] * base ** (-2.0 * np.arange(half) / d)[None, :]
-    c, s = np.cos(ang), np.sin(ang)
-    a, b = x[:, :half], x[:, half:]
-    return np.concatenate([a * c - b * s, b * c + a * s], 1)
+from tests.harness import bf16_round as _bf16
+from tests.harness import rope_rows as _rope_np
 
 
 def _floor(orc, L, lognormal, seed, heads):
@@ -114,3 +104,13 @@ def test_lognormal_norms_exceed_the_flat_bounds_by_rounding_alone(oracle_mod, L,
     assert e["o_scaled"] <= FLAT_ABS / 2, e
     assert e["lse_scaled"] <= LSE_ABS / 2, e
     assert e["o_lat_rel"] < REL and e["o_rel"] < REL, e
+
+
+def test_lognormal_rounding_alone_can_exceed_the_relative_bound(oracle_mod):
+    """Seed 64 of the same recipe (3000 tokens, all heads): rounding alone moves o_lat and o
+    by more than 4e-3 in relative L2.  So on log-normal norms the relative bound is applied to
+    the kernel's own error, against the oracle on the rounded operands (the `rounded` result
+    here, tests/harness.rounded_operand_ref in the GPU tests)."""
+    e = _errors(*_floor(oracle_mod, 3000, True, 64, range(128)))
+    assert e["o_lat_rel"] > REL and e["o_rel"] > REL, e
+    assert e["o_lat_scaled"] <= FLAT_ABS and e["lse_scaled"] <= LSE_ABS, e
