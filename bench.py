@@ -48,7 +48,7 @@ FLUSH_BYTES = 512 << 20
 # same workload and build (`ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum -k
 # regex:decode_tc_kernel -s 2 -c 1 python bench.py --plain-steps 3 --batch 16`, caches flushed
 # before the launch as in the timed loop).  None where no capture of that workload exists.
-DECODE_TRAFFIC = {"v3": 78050048 + 2524160}
+DECODE_TRAFFIC = {"v3": 78016512 + 2603520}
 
 
 def make_workload(name: str, batch: int | None = None):
