@@ -262,8 +262,9 @@ def peaks_of():
         return 6650.0, 1590.0, "fallback"
 
 
-STEP_CALLS = {True: "mla_cache_append, mla_absorb_q, mla_decode_project",
-              False: "mla_cache_append, mla_absorb_q, mla_decode, mla_out_proj"}
+def step_calls(front_fused: bool, project: bool) -> str:
+    front = "mla_append_absorb" if front_fused else "mla_cache_append, mla_absorb_q"
+    return front + (", mla_decode_project" if project else ", mla_decode, mla_out_proj")
 
 
 def fused_applies(wl) -> bool:
@@ -273,7 +274,8 @@ def fused_applies(wl) -> bool:
     return (d.n_h, d.d_h, d.d_c, d.d_r, d.page) == (128, 128, 512, 64, 64) and wl.act_dtype == "bf16"
 
 
-def measure(name, K, warmup, world, dev, clock_warmup_s, with_clock=True, project=False):
+def measure(name, K, warmup, world, dev, clock_warmup_s, with_clock=True, project=False, separate_front=False,
+            out_f32=False):
     """Time one workload: K steps of the whole path (CUDA graph, L2 flushed before each step),
     K decode-only replays, K end-to-end steps from pinned host buffers.  Returns a dict (device
     times already reduced to the max over ranks) and the workload."""
@@ -296,22 +298,32 @@ def measure(name, K, warmup, world, dev, clock_warmup_s, with_clock=True, projec
     q_abs = torch.empty((T, wl.dims.n_h, wl.dims.row), dtype=run.q_c.dtype, device=dev)
     o_lat = torch.empty((T, wl.dims.n_h, wl.dims.d_c), dtype=torch.float32, device=dev)
     lse = torch.empty((T, wl.dims.n_h), dtype=torch.float32, device=dev)
-    o = torch.empty((T, wl.dims.n_h, wl.dims.d_h), dtype=torch.float32, device=dev)
+    # the layer output in the activation dtype (bf16 on every V3 workload, fp32 for the toy)
+    out_dt = "bf16" if (wl.act_dtype == "bf16" and not out_f32) else "f32"
+    o = torch.empty((T, wl.dims.n_h, wl.dims.d_h), dtype=torch.bfloat16 if out_dt == "bf16" else torch.float32,
+                    device=dev)
     L.workspace(B, s_q, run.max_seq_len)
     decode_launches = 2  # split-KV main kernel + log-sum-exp combine
     fused = fused_applies(wl) and project
-    # append + absorb + (main + fused merge/projection | main + combine + out_proj)
-    launches_per_step = 1 + 1 + (2 if fused else decode_launches + 1)
+    # append + absorb: one launch through mla_append_absorb where the tensor-core absorption
+    # applies (the fused_applies shape), else two
+    front = 1 if (fused_applies(wl) and not separate_front) else 2
+    # + (main + fused merge/projection | main + combine + out_proj)
+    launches_per_step = front + (2 if fused else decode_launches + 1)
 
     def step(_unused=None, tok=(tok_seq, tok_pos, c_new, k_new), qin=(run.q_c, run.q_r, run.q_pos), out=o):
-        L.append(run.cache, tok[2], tok[3], tok[0], tok[1], run.block_table)
-        L.absorb(qin[0], qin[1], qin[2], out=q_abs)
+        if separate_front:
+            L.append(run.cache, tok[2], tok[3], tok[0], tok[1], run.block_table)
+            L.absorb(qin[0], qin[1], qin[2], out=q_abs)
+        else:
+            L.append_absorb(run.cache, tok[2], tok[3], tok[0], tok[1], run.block_table, qin[0], qin[1], qin[2],
+                            out=q_abs)
         if fused:
-            L.decode_project(run.cache, q_abs, run.block_table, run.seq_lens, s_q, run.max_seq_len, "f32",
+            L.decode_project(run.cache, q_abs, run.block_table, run.seq_lens, s_q, run.max_seq_len, out_dt,
                              o=out, o_lat=o_lat, lse=lse)
         else:
             L.decode(run.cache, q_abs, run.block_table, run.seq_lens, s_q, run.max_seq_len, o_lat=o_lat, lse=lse)
-            L.out_proj(o_lat, "f32", out=out)
+            L.out_proj(o_lat, out_dt, out=out)
 
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(device=dev)
@@ -407,6 +419,7 @@ def measure(name, K, warmup, world, dev, clock_warmup_s, with_clock=True, projec
         raise SystemExit(f"device error during the timed region ({name})")
     del g_step, g_dec, g_e2e
     res = dict(step_ms=step_ms, dec_ms=dec_ms, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, fused=fused,
+               calls=step_calls(front == 1, fused),
                launches=(launches_per_step + decode_launches) * K, clocks=clk.summary() if with_clock else None)
     del run, flush, h_pack, d_pack, h_out
     torch.cuda.synchronize()
@@ -531,7 +544,8 @@ def run_mine(args):
         dist.barrier()
 
     K = args.steps
-    r, wl = measure(args.config, K, args.warmup, world, dev, args.clock_warmup_s, project=args.project)
+    r, wl = measure(args.config, K, args.warmup, world, dev, args.clock_warmup_s, project=args.project,
+                    separate_front=args.separate_front, out_f32=args.out_f32)
     rf = roofline_of(wl, r["dec_ms"])
     tokens = job_tokens(wl.T, world)
     line = None
@@ -545,7 +559,7 @@ def run_mine(args):
                        "context": int(wl.seq_lens.max()), "parallelism": f"replicas x{world}",
                        "l2": "flushed before every timed step (512 MiB write outside the events)",
                        "launch": "each step is one CUDA-graph replay of the calls",
-                       "calls": STEP_CALLS[r["fused"]]},
+                       "calls": r["calls"]},
             "decode": {"kernel": "mla_decode (tcgen05 split-KV main with in-kernel schedule + LSE combine)",
                        "ms": r["dec_ms"], "tokens_per_s": tokens / (r["dec_ms"] * 1e-3), "cache_gbs": rf["gbs"],
                        "tflops": rf["tfl"], "frac_hbm": rf["gbs"] / rf["hbm_peak"],
@@ -571,10 +585,11 @@ def run_mine(args):
         for name in WORKLOADS:
             if name == args.config:
                 continue
-            r2, wl2 = measure(name, k2, args.warmup, world, dev, 0.8, project=args.project)
+            r2, wl2 = measure(name, k2, args.warmup, world, dev, 0.8, project=args.project,
+                              separate_front=args.separate_front, out_f32=args.out_f32)
             rf2 = roofline_of(wl2, r2["dec_ms"])
             t2 = job_tokens(wl2.T, world)
-            c = {"workload": WORKLOADS[name], "steps": k2, "step_ms": r2["step_ms"], "calls": STEP_CALLS[r2["fused"]],
+            c = {"workload": WORKLOADS[name], "steps": k2, "step_ms": r2["step_ms"], "calls": r2["calls"],
                  "tokens_per_s": t2 / (r2["step_ms"] * 1e-3),
                  "decode_ms": r2["dec_ms"], "decode_tokens_per_s": t2 / (r2["dec_ms"] * 1e-3),
                  "cache_gbs": rf2["gbs"], "tflops": rf2["tfl"], "frac_hbm": rf2["gbs"] / rf2["hbm_peak"],
@@ -646,6 +661,10 @@ def main():
     ap.add_argument("--prefill-lens", default=None, help="with --prefill-only: comma-separated prompt lengths")
     ap.add_argument("--plain-project", action="store_true",
                     help="with --plain-steps: steps through mla_decode_project")
+    ap.add_argument("--out-f32", action="store_true", help="write the layer output o in fp32 (default: the "
+                                                              "activation dtype)")
+    ap.add_argument("--separate-front", action="store_true",
+                    help="step with mla_cache_append + mla_absorb_q instead of mla_append_absorb")
     ap.add_argument("--project", action="store_true",
                     help="step with mla_decode_project (fused merge + projection) instead of mla_decode + "
                          "mla_out_proj")

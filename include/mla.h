@@ -146,6 +146,25 @@ mla_status_t mla_cache_append(const mla_dims_t *dims, int T, const void *c_kv, c
                               mla_stream_t stream);
 
 /* ----------------------------------------------------------------------------------------
+ * mla_append_absorb -- mla_cache_append followed by mla_absorb_q, in one call.  The two
+ * write different buffers (the cache; q_abs) and neither reads the other's output, so where
+ * the tensor-core absorption applies (n_h any, d_h = 128, d_c = 512, d_r = 64, bf16
+ * activations, bf16 or FP8 cache, no MLA_FLAG_SIMT_PROJ, 16-byte aligned q_c, q_r, w_uk,
+ * q_abs) both run in ONE launch, the cache writes overlapping the absorption's weight fetch;
+ * elsewhere the two are launched one after the other.  The results are bit for bit those of
+ * the two calls.
+ *   Arguments: those of mla_cache_append (T_new new tokens, pos_new their positions), then
+ *   those of mla_absorb_q (T query tokens, pos their positions).
+ * Errors: those of either call, checked before anything is launched.
+ * ---------------------------------------------------------------------------------------- */
+mla_status_t mla_append_absorb(const mla_dims_t *dims, int T_new, const void *c_kv, const void *k_r,
+                               const int32_t *seq_idx, const int32_t *pos_new,
+                               const int32_t *block_table, int num_seqs, int max_blocks_per_seq,
+                               int num_blocks, void *kv_pool, void *kr_pool, float *kv_scale, int T,
+                               const void *q_c, const void *q_r, const int32_t *pos, const void *w_uk,
+                               void *q_abs, mla_stream_t stream);
+
+/* ----------------------------------------------------------------------------------------
  * mla_decode_workspace_size -- bytes of device workspace mla_decode needs for B sequences of
  * s_q queries each and sequence lengths up to max_seq_len, on the current device.  Returns 0
  * for invalid arguments or when the current device cannot be queried.

@@ -8,9 +8,7 @@
 // One warp per token.  The work is a few KB per token, bound by its HBM writes; the only
 // arithmetic is the RoPE rotation (angle in fp64) and, for FP8, a warp max and the e4m3
 // conversion (cvt.rn.satfinite through cuda_fp8.h).
-#include <float.h>
-
-#include "mla_internal.cuh"
+#include "append_body.cuh"
 
 namespace mla {
 namespace {
@@ -19,78 +17,38 @@ constexpr int kWarpsPerBlock = 8;
 
 template <typename Tin, int KV>  // KV: 0 = f32 cache, 1 = bf16 cache, 2 = fp8 content cache
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
-append_kernel(int T, int d_c, int d_r, int page, const __grid_constant__ RopeFreqs rope, const Tin *__restrict__ c_kv,
-              const Tin *__restrict__ k_r, const int32_t *__restrict__ seq_idx,
-              const int32_t *__restrict__ pos, const int32_t *__restrict__ bt, int num_seqs,
-              int max_blocks, int num_blocks, void *kv_pool, __nv_bfloat16 *kr_pool,
-              float *kv_scale, unsigned *err) {
+append_kernel(const __grid_constant__ AppendArgs a, const __grid_constant__ RopeFreqs rope, unsigned *err) {
     // The query absorption that usually follows may start now: it waits for this kernel on the
     // device before it reads anything that could depend on it.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
-    if (t >= T) return;
-    const int s = seq_idx[t];
-    const int p = pos[t];
-    if (s < 0 || s >= num_seqs || p < 0 || p / page >= max_blocks) {
-        if (lane == 0) record_error(err, kErrBadBlock);
-        return;
-    }
-    const int blk = bt[(size_t)s * max_blocks + p / page];
-    if (blk < 0 || blk >= num_blocks) {
-        if (lane == 0) record_error(err, kErrBadBlock);
-        return;
-    }
-    const size_t slot = (size_t)blk * page + (p % page);
-    const Tin *c_in = c_kv + (size_t)t * d_c;
-    const Tin *k_in = k_r + (size_t)t * d_r;
-
-    // RoPE of the shared key (pairs k, k + d_r/2).
-    const int half = d_r >> 1;
-    for (int k = lane; k < half; k += 32) {
-        float cs, sn;
-        rope_cos_sin(rope, k, p, &cs, &sn);
-        float x0 = to_f32(k_in[k]), x1 = to_f32(k_in[k + half]);
-        float y0 = x0 * cs - x1 * sn;
-        float y1 = x1 * cs + x0 * sn;
-        if (KV == 0) {
-            float *row = reinterpret_cast<float *>(kv_pool) + slot * (d_c + d_r) + d_c;
-            row[k] = y0;
-            row[k + half] = y1;
-        } else if (KV == 1) {
-            __nv_bfloat16 *row = reinterpret_cast<__nv_bfloat16 *>(kv_pool) + slot * (d_c + d_r) + d_c;
-            row[k] = __float2bfloat16_rn(y0);
-            row[k + half] = __float2bfloat16_rn(y1);
-        } else {
-            __nv_bfloat16 *row = kr_pool + slot * d_r;
-            row[k] = __float2bfloat16_rn(y0);
-            row[k + half] = __float2bfloat16_rn(y1);
-        }
-    }
-
-    if (KV == 0) {
-        float *row = reinterpret_cast<float *>(kv_pool) + slot * (d_c + d_r);
-        for (int k = lane; k < d_c; k += 32) row[k] = to_f32(c_in[k]);
-    } else if (KV == 1) {
-        __nv_bfloat16 *row = reinterpret_cast<__nv_bfloat16 *>(kv_pool) + slot * (d_c + d_r);
-        for (int k = lane; k < d_c; k += 32) row[k] = __float2bfloat16_rn(to_f32(c_in[k]));
-    } else {
-        float amax = 0.f;
-        for (int k = lane; k < d_c; k += 32) amax = fmaxf(amax, fabsf(to_f32(c_in[k])));
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        float sc = 1.f;
-        if (amax > 0.f) sc = fmaxf(__fdiv_rn(amax, 448.f), FLT_MIN);
-        uint8_t *row = reinterpret_cast<uint8_t *>(kv_pool) + slot * d_c;
-        for (int k = lane; k < d_c; k += 32) {
-            float x = __fdiv_rn(to_f32(c_in[k]), sc);
-            row[k] = (uint8_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
-        }
-        if (lane == 0) kv_scale[slot] = sc;
-    }
+    if (t >= a.T) return;
+    append_token<Tin, KV>(a, rope, t, threadIdx.x & 31, err);
 }
 
 }  // namespace
+
+AppendArgs append_args(const mla_dims_t &d, int T, const void *c_kv, const void *k_r, const int32_t *seq_idx,
+                       const int32_t *pos, const int32_t *bt, int num_seqs, int max_blocks, int num_blocks,
+                       void *kv_pool, void *kr_pool, float *kv_scale) {
+    AppendArgs a;
+    a.T = T;
+    a.d_c = d.d_c;
+    a.d_r = d.d_r;
+    a.page = d.page_size;
+    a.c_kv = c_kv;
+    a.k_r = k_r;
+    a.seq_idx = seq_idx;
+    a.pos = pos;
+    a.bt = bt;
+    a.num_seqs = num_seqs;
+    a.max_blocks = max_blocks;
+    a.num_blocks = num_blocks;
+    a.kv_pool = kv_pool;
+    a.kr_pool = reinterpret_cast<__nv_bfloat16 *>(kr_pool);
+    a.kv_scale = kv_scale;
+    return a;
+}
 
 cudaError_t launch_append(const mla_dims_t &d, int T, const void *c_kv, const void *k_r,
                           const int32_t *seq_idx, const int32_t *pos, const int32_t *bt,
@@ -100,12 +58,9 @@ cudaError_t launch_append(const mla_dims_t &d, int T, const void *c_kv, const vo
     dim3 grid((T + kWarpsPerBlock - 1) / kWarpsPerBlock), block(kWarpsPerBlock * 32);
     const RopeFreqs rope = make_rope_freqs((double)d.rope_base, d.d_r);
     unsigned *err = device_error_word();
-    auto *krp = reinterpret_cast<__nv_bfloat16 *>(kr_pool);
-#define MLA_APPEND(TIN, KV)                                                                       \
-    append_kernel<TIN, KV><<<grid, block, 0, st>>>(                                                \
-        T, d.d_c, d.d_r, d.page_size, rope, reinterpret_cast<const TIN *>(c_kv),    \
-        reinterpret_cast<const TIN *>(k_r), seq_idx, pos, bt, num_seqs, max_blocks, num_blocks,    \
-        kv_pool, krp, kv_scale, err)
+    const AppendArgs a = append_args(d, T, c_kv, k_r, seq_idx, pos, bt, num_seqs, max_blocks, num_blocks, kv_pool,
+                                     kr_pool, kv_scale);
+#define MLA_APPEND(TIN, KV) append_kernel<TIN, KV><<<grid, block, 0, st>>>(a, rope, err)
     const bool in_bf16 = d.act_dtype == MLA_DTYPE_BF16;
     switch (d.kv_dtype) {
         case MLA_DTYPE_F32:

@@ -5,6 +5,7 @@
 #include <mutex>
 #include <stdio.h>
 
+#include "append_body.cuh"
 #include "mla_internal.cuh"
 
 namespace mla {
@@ -110,22 +111,34 @@ mla_status_t mla_get_last_device_error(void) {
     return (mla_status_t)v;
 }
 
-mla_status_t mla_absorb_q(const mla_dims_t *dims, int T, const void *q_c, const void *q_r,
-                          const int32_t *pos, const void *w_uk, void *q_abs,
-                          mla_stream_t stream) {
+// Host checks of mla_absorb_q (MLA_OK with *work = false: nothing to do).
+static mla_status_t check_absorb(const mla_dims_t *dims, int T, const void *q_c, const void *q_r,
+                                 const int32_t *pos, const void *w_uk, void *q_abs, bool *work) {
+    *work = false;
     mla_status_t s = check_dims(dims);
     if (s != MLA_OK) return s;
     if (T < 0) return MLA_ERR_INVALID_ARG;
     if (T == 0) return MLA_OK;
     if (!q_c || !q_r || !pos || !w_uk || !q_abs) return MLA_ERR_INVALID_ARG;
+    *work = true;
+    return MLA_OK;
+}
+
+mla_status_t mla_absorb_q(const mla_dims_t *dims, int T, const void *q_c, const void *q_r,
+                          const int32_t *pos, const void *w_uk, void *q_abs,
+                          mla_stream_t stream) {
+    bool work;
+    mla_status_t s = check_absorb(dims, T, q_c, q_r, pos, w_uk, q_abs, &work);
+    if (s != MLA_OK || !work) return s;
     return from_cuda(launch_absorb_q(*dims, T, q_c, q_r, pos, w_uk, q_abs, (cudaStream_t)stream));
 }
 
-mla_status_t mla_cache_append(const mla_dims_t *dims, int T, const void *c_kv, const void *k_r,
-                              const int32_t *seq_idx, const int32_t *pos,
-                              const int32_t *block_table, int num_seqs, int max_blocks_per_seq,
-                              int num_blocks, void *kv_pool, void *kr_pool, float *kv_scale,
-                              mla_stream_t stream) {
+// Host checks of mla_cache_append.
+static mla_status_t check_append(const mla_dims_t *dims, int T, const void *c_kv, const void *k_r,
+                                 const int32_t *seq_idx, const int32_t *pos, const int32_t *block_table,
+                                 int num_seqs, int max_blocks_per_seq, int num_blocks, void *kv_pool,
+                                 void *kr_pool, float *kv_scale, bool *work) {
+    *work = false;
     mla_status_t s = check_dims(dims);
     if (s != MLA_OK) return s;
     if (T < 0 || num_seqs < 0 || max_blocks_per_seq < 0 || num_blocks < 0) return MLA_ERR_INVALID_ARG;
@@ -135,9 +148,50 @@ mla_status_t mla_cache_append(const mla_dims_t *dims, int T, const void *c_kv, c
     if ((int64_t)max_blocks_per_seq * dims->page_size > INT_MAX) return MLA_ERR_INVALID_ARG;
     const bool fp8 = dims->kv_dtype == MLA_DTYPE_FP8_E4M3;
     if (fp8 != (kr_pool != nullptr) || fp8 != (kv_scale != nullptr)) return MLA_ERR_INVALID_ARG;
+    *work = true;
+    return MLA_OK;
+}
+
+mla_status_t mla_cache_append(const mla_dims_t *dims, int T, const void *c_kv, const void *k_r,
+                              const int32_t *seq_idx, const int32_t *pos,
+                              const int32_t *block_table, int num_seqs, int max_blocks_per_seq,
+                              int num_blocks, void *kv_pool, void *kr_pool, float *kv_scale,
+                              mla_stream_t stream) {
+    bool work;
+    mla_status_t s = check_append(dims, T, c_kv, k_r, seq_idx, pos, block_table, num_seqs, max_blocks_per_seq,
+                                  num_blocks, kv_pool, kr_pool, kv_scale, &work);
+    if (s != MLA_OK || !work) return s;
     return from_cuda(launch_append(*dims, T, c_kv, k_r, seq_idx, pos, block_table, num_seqs,
                                    max_blocks_per_seq, num_blocks, kv_pool, kr_pool, kv_scale,
                                    (cudaStream_t)stream));
+}
+
+mla_status_t mla_append_absorb(const mla_dims_t *dims, int T_new, const void *c_kv, const void *k_r,
+                               const int32_t *seq_idx, const int32_t *pos_new, const int32_t *block_table,
+                               int num_seqs, int max_blocks_per_seq, int num_blocks, void *kv_pool,
+                               void *kr_pool, float *kv_scale, int T, const void *q_c, const void *q_r,
+                               const int32_t *pos, const void *w_uk, void *q_abs, mla_stream_t stream) {
+    bool wa, wq;
+    mla_status_t s = check_append(dims, T_new, c_kv, k_r, seq_idx, pos_new, block_table, num_seqs,
+                                  max_blocks_per_seq, num_blocks, kv_pool, kr_pool, kv_scale, &wa);
+    if (s != MLA_OK) return s;
+    s = check_absorb(dims, T, q_c, q_r, pos, w_uk, q_abs, &wq);
+    if (s != MLA_OK) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    // one launch where the tensor-core absorption applies (the conditions of launch_absorb_q)
+    if (wa && wq && append_absorb_tc_supported(*dims) && !(dims->flags & MLA_FLAG_SIMT_PROJ) &&
+        aligned(q_c, 16) && aligned(q_r, 16) && aligned(w_uk, 16) && aligned(q_abs, 16)) {
+        const AppendArgs job = append_args(*dims, T_new, c_kv, k_r, seq_idx, pos_new, block_table, num_seqs,
+                                           max_blocks_per_seq, num_blocks, kv_pool, kr_pool, kv_scale);
+        return from_cuda(launch_append_absorb_tc(*dims, job, T, q_c, q_r, pos, w_uk, q_abs, st));
+    }
+    if (wa) {
+        s = from_cuda(launch_append(*dims, T_new, c_kv, k_r, seq_idx, pos_new, block_table, num_seqs,
+                                    max_blocks_per_seq, num_blocks, kv_pool, kr_pool, kv_scale, st));
+        if (s != MLA_OK) return s;
+    }
+    if (wq) return from_cuda(launch_absorb_q(*dims, T, q_c, q_r, pos, w_uk, q_abs, st));
+    return MLA_OK;
 }
 
 static bool use_tc(const mla_dims_t *d) {

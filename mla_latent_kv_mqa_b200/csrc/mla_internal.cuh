@@ -92,6 +92,12 @@ cudaError_t launch_absorb_q_tc(const mla_dims_t &d, int T, const void *q_c, cons
 cudaError_t launch_out_proj_tc(const mla_dims_t &d, int T, const float *o_lat, const void *w_uv, void *o,
                                mla_dtype_t out_dtype, cudaStream_t st);
 
+// mla_cache_append + mla_absorb_q in one launch (tensor-core absorption, bf16 or FP8 cache).
+struct AppendArgs;
+bool append_absorb_tc_supported(const mla_dims_t &d);
+cudaError_t launch_append_absorb_tc(const mla_dims_t &d, const AppendArgs &job, int T, const void *q_c,
+                                    const void *q_r, const int32_t *pos, const void *w_uk, void *q_abs,
+                                    cudaStream_t st);
 // CUDA-core split-KV decode.  Splits every query row into n_split segments of seg_len tokens.
 struct SimtPlan {
     int n_split;

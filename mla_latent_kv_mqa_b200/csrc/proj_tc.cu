@@ -18,6 +18,7 @@
 // in TMEM, and the epilogue writes straight from tcgen05.ld.
 #include <math.h>
 
+#include "append_body.cuh"
 #include "mla_internal.cuh"
 #include "sm100.cuh"
 #include "tmap.cuh"
@@ -409,11 +410,24 @@ constexpr int AB_DATA = AB_B + 2 * TN * 128;      // + 32 KB
 constexpr int AB_SMEM = 1024 + AB_DATA + 256;
 static_assert(TN * DCL * 2 <= NWB * WBOX, "the result tile reuses the weight region");
 
+// KV >= 0: the same launch also appends job.T new tokens to the cache (mla_cache_append's
+// work, KV as in append_token: 1 = bf16 cache, 2 = fp8 content cache) in extra CTAs
+// blockIdx.x >= n_h of the first token tile, one warp per token; their work is independent
+// of the absorption, so it overlaps the absorption's weight fetch instead of preceding it.
+template <int KV>
 __global__ void __launch_bounds__(128, 1)
 absorb_tc_kernel(const __grid_constant__ CUtensorMap tm_w, int T, int n_h, const __grid_constant__ RopeFreqs rope,
                  const __nv_bfloat16 *__restrict__ q_c, const __nv_bfloat16 *__restrict__ q_r,
-                 const int32_t *__restrict__ pos, __nv_bfloat16 *__restrict__ q_abs, unsigned *err) {
+                 const int32_t *__restrict__ pos, __nv_bfloat16 *__restrict__ q_abs, unsigned *err,
+                 const __grid_constant__ AppendArgs job) {
     pdl_trigger();  // the decode that follows may set itself up (it waits for q_abs on the device)
+    if (KV >= 0 && (int)blockIdx.x >= n_h) {  // an append CTA
+        if (blockIdx.y != 0) return;
+        pdl_wait();  // the new tokens may be the previous kernel's output
+        const int t = ((int)blockIdx.x - n_h) * 4 + (threadIdx.x >> 5);
+        if (t < job.T) append_token<__nv_bfloat16, (KV < 0 ? 1 : KV)>(job, rope, t, threadIdx.x & 31, err);
+        return;
+    }
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_u32(smem_raw);
     const uint32_t data_s = (raw_s + 1023u) & ~1023u;
@@ -584,10 +598,32 @@ cudaError_t launch_absorb_q_tc(const mla_dims_t &d, int T, const void *q_c, cons
                                const int32_t *pos, const void *w_uk, void *q_abs, cudaStream_t st) {
     CUtensorMap tm;
     if (!tmap_bf16_2d(&tm, w_uk, DCL, (uint64_t)d.n_h * DH, DCL * 2, 64, 128)) return cudaErrorInvalidValue;
-    return launch_dependent(absorb_tc_kernel, dim3(d.n_h, (T + TN - 1) / TN), AB_SMEM, st, tm, T, d.n_h,
+    AppendArgs none = {};
+    return launch_dependent(absorb_tc_kernel<-1>, dim3(d.n_h, (T + TN - 1) / TN), AB_SMEM, st, tm, T, d.n_h,
                             make_rope_freqs((double)d.rope_base, d.d_r), reinterpret_cast<const __nv_bfloat16 *>(q_c),
                             reinterpret_cast<const __nv_bfloat16 *>(q_r), pos,
-                            reinterpret_cast<__nv_bfloat16 *>(q_abs), device_error_word());
+                            reinterpret_cast<__nv_bfloat16 *>(q_abs), device_error_word(), none);
+}
+
+bool append_absorb_tc_supported(const mla_dims_t &d) {
+    return proj_tc_supported(d) && (d.kv_dtype == MLA_DTYPE_BF16 || d.kv_dtype == MLA_DTYPE_FP8_E4M3);
+}
+
+cudaError_t launch_append_absorb_tc(const mla_dims_t &d, const AppendArgs &job, int T, const void *q_c,
+                                    const void *q_r, const int32_t *pos, const void *w_uk, void *q_abs,
+                                    cudaStream_t st) {
+    CUtensorMap tm;
+    if (!tmap_bf16_2d(&tm, w_uk, DCL, (uint64_t)d.n_h * DH, DCL * 2, 64, 128)) return cudaErrorInvalidValue;
+    const dim3 grid(d.n_h + (job.T + 3) / 4, (T + TN - 1) / TN);
+    const RopeFreqs rope = make_rope_freqs((double)d.rope_base, d.d_r);
+    auto qc = reinterpret_cast<const __nv_bfloat16 *>(q_c);
+    auto qr = reinterpret_cast<const __nv_bfloat16 *>(q_r);
+    auto qa = reinterpret_cast<__nv_bfloat16 *>(q_abs);
+    if (d.kv_dtype == MLA_DTYPE_FP8_E4M3)
+        return launch_dependent(absorb_tc_kernel<2>, grid, AB_SMEM, st, tm, T, d.n_h, rope, qc, qr, pos, qa,
+                                device_error_word(), job);
+    return launch_dependent(absorb_tc_kernel<1>, grid, AB_SMEM, st, tm, T, d.n_h, rope, qc, qr, pos, qa,
+                            device_error_word(), job);
 }
 
 cudaError_t launch_out_proj_tc(const mla_dims_t &d, int T, const float *o_lat, const void *w_uv, void *o,

@@ -89,6 +89,19 @@ class MLADecodeLayer:
         N.mla_absorb_q(d, T, q_c, q_r, pos, self.w_uk, out, stream)
         return out
 
+    def append_absorb(self, cache: PagedLatentCache, c_kv, k_r, seq_idx, pos_new, block_table, q_c, q_r, pos,
+                      out=None, stream=None):
+        """append then absorb in one library call; returns q_abs."""
+        T_new = c_kv.shape[0]
+        B, max_blocks = block_table.shape
+        T = q_c.shape[0]
+        d = self.dims
+        if out is None:
+            out = torch.empty((T, d.n_h, d.d_c + d.d_r), dtype=TORCH_ACT[d.act_dtype], device=self.device)
+        N.mla_append_absorb(d, T_new, c_kv, k_r, seq_idx, pos_new, block_table, B, max_blocks, cache.num_blocks,
+                            cache.kv_pool, cache.kr_pool, cache.kv_scale, T, q_c, q_r, pos, self.w_uk, out, stream)
+        return out
+
     def workspace(self, B, s_q, max_seq_len):
         key = (B, s_q, max_seq_len)
         if self._ws_key != key:

@@ -68,6 +68,8 @@ _lib.mla_decode.argtypes = [_dp, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _
 _lib.mla_decode_fixed_scratch.argtypes = [_dp, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _i,
                                           _vp, _vp, _vp]
 _lib.mla_out_proj.argtypes = [_dp, _i, _vp, _vp, _vp, _i, _vp]
+_lib.mla_append_absorb.argtypes = [_dp, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp,
+                                   _vp, _vp, _vp]
 _lib.mla_decode_project.argtypes = [_dp, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _i, _vp, _sz,
                                     _vp, _vp, _i, _vp, _vp, _vp]
 _lib.mla_prefill_workspace_size.argtypes = [_dp, _i]
@@ -80,7 +82,8 @@ _lib.mla_status_string.argtypes = [_i]
 _lib.mla_status_string.restype = ctypes.c_char_p
 _lib.mla_version.restype = _i
 for _f in ("mla_absorb_q", "mla_cache_append", "mla_decode", "mla_decode_fixed_scratch", "mla_out_proj",
-           "mla_decode_project", "mla_prefill", "mla_get_last_device_error", "mla_lse_merge_prepare",
+           "mla_decode_project", "mla_prefill", "mla_append_absorb", "mla_get_last_device_error",
+           "mla_lse_merge_prepare",
            "mla_lse_merge_finish"):
     getattr(_lib, _f).restype = _i
 
@@ -137,6 +140,15 @@ def mla_cache_append(dims, T, c_kv, k_r, seq_idx, pos, block_table, num_seqs, ma
                                  _ptr(pos), _ptr(block_table), num_seqs, max_blocks_per_seq,
                                  num_blocks, _ptr(kv_pool), _ptr(kr_pool), _ptr(kv_scale),
                                  _stream(stream)), "mla_cache_append")
+
+
+def mla_append_absorb(dims, T_new, c_kv, k_r, seq_idx, pos_new, block_table, num_seqs, max_blocks_per_seq,
+                      num_blocks, kv_pool, kr_pool, kv_scale, T, q_c, q_r, pos, w_uk, q_abs, stream=None):
+    """mla_cache_append then mla_absorb_q (one launch where the tensor-core absorption applies)."""
+    _check(_lib.mla_append_absorb(ctypes.byref(dims), T_new, _ptr(c_kv), _ptr(k_r), _ptr(seq_idx), _ptr(pos_new),
+                                  _ptr(block_table), num_seqs, max_blocks_per_seq, num_blocks, _ptr(kv_pool),
+                                  _ptr(kr_pool), _ptr(kv_scale), T, _ptr(q_c), _ptr(q_r), _ptr(pos), _ptr(w_uk),
+                                  _ptr(q_abs), _stream(stream)), "mla_append_absorb")
 
 
 def mla_decode_workspace_size(dims, B, s_q, max_seq_len) -> int:

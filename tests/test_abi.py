@@ -88,6 +88,14 @@ def test_host_argument_checks(N):
     assert dp_call(q_abs=None) == N.MLA_ERR_INVALID_ARG
     assert dp_call(out_dtype=N.MLA_DTYPE_FP8_E4M3) == N.MLA_ERR_UNSUPPORTED
     assert dp_call(B=0, w_uv=None) == N.MLA_OK
+    # append + absorb in one call: each part's checks, before anything is launched
+    def aa(T_new=4, c_kv=16, T=4, q_c=16, kr=None):
+        return L.mla_append_absorb(dp, T_new, c_kv, 16, 16, 16, 16, 2, 4, 8, 16, kr, None, T, q_c, 16, 16, 16, 16,
+                                   None)
+    assert aa(c_kv=None) == N.MLA_ERR_INVALID_ARG and aa(q_c=None) == N.MLA_ERR_INVALID_ARG
+    assert aa(T_new=-1) == N.MLA_ERR_INVALID_ARG and aa(T=-1) == N.MLA_ERR_INVALID_ARG
+    assert aa(kr=16) == N.MLA_ERR_INVALID_ARG  # a RoPE pool only with the FP8 cache
+    assert aa(T_new=0, c_kv=None, T=0, q_c=None) == N.MLA_OK
     # prefill: the supported shape, sizes, null and misaligned pointers, workspace size
     def pf(B=2, T=256, max_len=128, cu=16, q_c=16, o=16, ws=256, ws_bytes=1 << 40, d=dp):
         return L.mla_prefill(d, B, cu, T, max_len, q_c, 16, 16, 16, 16, 16, ws, ws_bytes, o, None, None)
