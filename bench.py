@@ -275,7 +275,7 @@ def fused_applies(wl) -> bool:
 
 
 def measure(name, K, warmup, world, dev, clock_warmup_s, with_clock=True, project=False, separate_front=False,
-            out_f32=False):
+            out_f32=False, fp8_mma=False):
     """Time one workload: K steps of the whole path (CUDA graph, L2 flushed before each step),
     K decode-only replays, K end-to-end steps from pinned host buffers.  Returns a dict (device
     times already reduced to the max over ranks) and the workload."""
@@ -285,7 +285,8 @@ def measure(name, K, warmup, world, dev, clock_warmup_s, with_clock=True, projec
     from tests.harness import GpuRun
 
     wl = make_workload(name)
-    run = GpuRun(wl, dev=dev)
+    flags = N.MLA_FLAG_FP8_MMA if (fp8_mma and wl.kv_dtype == "fp8") else 0
+    run = GpuRun(wl, dev=dev, flags=flags)
     run.fill_cache()
     L = run.layer
     B, s_q, T = wl.B, wl.s_q, wl.T
@@ -545,7 +546,7 @@ def run_mine(args):
 
     K = args.steps
     r, wl = measure(args.config, K, args.warmup, world, dev, args.clock_warmup_s, project=args.project,
-                    separate_front=args.separate_front, out_f32=args.out_f32)
+                    separate_front=args.separate_front, out_f32=args.out_f32, fp8_mma=args.fp8_mma)
     rf = roofline_of(wl, r["dec_ms"])
     tokens = job_tokens(wl.T, world)
     line = None
@@ -586,7 +587,7 @@ def run_mine(args):
             if name == args.config:
                 continue
             r2, wl2 = measure(name, k2, args.warmup, world, dev, 0.8, project=args.project,
-                              separate_front=args.separate_front, out_f32=args.out_f32)
+                              separate_front=args.separate_front, out_f32=args.out_f32, fp8_mma=args.fp8_mma)
             rf2 = roofline_of(wl2, r2["dec_ms"])
             t2 = job_tokens(wl2.T, world)
             c = {"workload": WORKLOADS[name], "steps": k2, "step_ms": r2["step_ms"], "calls": r2["calls"],
@@ -661,6 +662,8 @@ def main():
     ap.add_argument("--prefill-lens", default=None, help="with --prefill-only: comma-separated prompt lengths")
     ap.add_argument("--plain-project", action="store_true",
                     help="with --plain-steps: steps through mla_decode_project")
+    ap.add_argument("--fp8-mma", action="store_true",
+                    help="FP8 cache: content scores on the FP8 tensor core (MLA_FLAG_FP8_MMA)")
     ap.add_argument("--out-f32", action="store_true", help="write the layer output o in fp32 (default: the "
                                                               "activation dtype)")
     ap.add_argument("--separate-front", action="store_true",

@@ -85,6 +85,16 @@ typedef enum {
 #define MLA_FLAG_SIMT_DECODE 1u /* run mla_decode on the CUDA-core kernel even where the
                                    tensor-core kernel applies (cross-checks) */
 #define MLA_FLAG_SIMT_PROJ 2u   /* same for mla_absorb_q and mla_out_proj */
+/* FP8 cache only: compute the content part of the scores on the FP8 tensor core
+ * (tcgen05 kind::f8f6f4) from the cached e4m3 codes as they are, instead of dequantising every
+ * page to bf16 first.  The absorbed query is split per head into two e4m3 parts,
+ * q_lat ~ alpha_h (hi + lo) with alpha_h = max|q_lat| / 448, hi = e4m3(q_lat / alpha_h),
+ * lo = e4m3(q_lat / alpha_h - hi) (about 7 significant bits, near bf16's 8), and the RoPE part
+ * runs in bf16 on (q_R / alpha_h) . (k_R / s_j), so each score is
+ *     s_j = alpha_h s_j [ (hi + lo) . c8_j + (q_R / alpha_h) . (k_R,j / s_j) ] / sqrt(d_h + d_R).
+ * The value product P . V keeps bf16 V (dequantised on chip).  QuantMLA review, Motivation
+ * & Problem Statement (an FP8 content cache next to a high-precision RoPE-key cache). */
+#define MLA_FLAG_FP8_MMA 8u
 #define MLA_FLAG_TEST_GIVE_UP 4u /* test of the failure path of the tensor-core decode: in
                                     every cluster with two or more pages, after the copies of
                                     the first page have started, one bounded wait (20 us) on a

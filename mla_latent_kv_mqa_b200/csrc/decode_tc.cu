@@ -50,6 +50,7 @@
 // MMAs waits (again bounded) for them, so no asynchronous write targets a CTA that has left.
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
+#include <float.h>
 #include <math.h>
 
 #include <mutex>
@@ -139,20 +140,34 @@ struct __align__(8) Ctrl {
     float lx[2][NH];            // QK CTA: the second softmax half's row sums, by segment parity
     float fac[2][NH];           // QK CTA: per-head rescale factors of a page, by page parity
 };
+// FP8 cache with the content scores on the FP8 tensor core (MM): per segment, the per-head
+// scale of the e4m3 query and the two halves' max |q_lat|; per page (ring of 3, by page count),
+// the tokens' scales times log2(e)/sqrt(d_h + d_R).
+struct Q8Extra {
+    float qalpha[NH];
+    float qamax[2][NH];
+    float pscale[3][PG];
+};
 // Shared-memory plan of the bf16 (F8 = false) and FP8 (F8 = true) kernels.  The FP8 QK CTA
-// keeps two page stages (its staging slots take the third).
-template <bool F8>
+// keeps two page stages, and its staging slots take the third; with MM = true the codes land
+// in the stage itself, so all three stages stay, followed by the Q8Extra block.
+template <bool F8, bool MM = false>
 struct Lay {
-    static constexpr int kv_stages = F8 ? 2 : KV_STAGES;
+    static constexpr int kv_stages = (F8 && !MM) ? 2 : KV_STAGES;
     static constexpr int stg_off = kv_stages * KV_STAGE;
-    static constexpr int data_a = stg_off + (F8 ? 2 * STG_SLOT : 0);
+    static constexpr int q8_off = stg_off;
+    static constexpr int data_a = stg_off + (F8 ? (MM ? (int)sizeof(Q8Extra) : 2 * STG_SLOT) : 0);
     static constexpr int vstg_off = DATA_B;
     static constexpr int data_b = DATA_B + (F8 ? 2 * VSTG_SLOT : 0);
     static constexpr int data = data_a > data_b ? data_a : data_b;
     static constexpr int smem = 1024 + data + (int)((sizeof(Ctrl) + 127) / 128 * 128);
 };
-static_assert(Lay<false>::smem <= 232448 && Lay<true>::smem <= 232448, "shared memory per block");
+static_assert(Lay<false>::smem <= 232448 && Lay<true>::smem <= 232448 && Lay<true, true>::smem <= 232448,
+              "shared memory per block");
 static_assert(Lay<true>::stg_off % 1024 == 0 && Lay<true>::vstg_off % 1024 == 0, "staging alignment");
+// MM page stage: content codes as 4 K-major SW128 blocks [64 tokens x 128 B] (blocks 0-3), the
+// tokens' scales at block 4, the RoPE keys (bf16, divided on chip by the token's scale) at block 8.
+constexpr int MM_SCALE_OFF = 4 * CB;
 
 struct Params {
     const int32_t *bt;
@@ -253,6 +268,23 @@ __device__ __forceinline__ void dequant8(uint32_t src, float sc, uint32_t dst) {
         o[k] = pack_bf16x2(f.x * sc, f.y * sc);
     }
     st_shared_v4(dst, o[0], o[1], o[2], o[3]);
+}
+
+// bf16 pair (low half first) -> two floats.
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+// Two floats -> two e4m3 codes (nearest even, saturating), x in the low byte.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float x, float y) {
+    unsigned short r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(y), "f"(x));
+    return r;
+}
+// Two e4m3 codes (low byte first) -> their exact values.
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t w) {
+    uint32_t hh;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hh) : "h"((unsigned short)w));
+    return __half22float2(*reinterpret_cast<const __half2 *>(&hh));
 }
 
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
@@ -423,11 +455,13 @@ constexpr int BAR_VCONV = 5;  // PV CTA: the FP8 converter warps
 // F8 = false: bf16 cache; tm_kv9 loads whole pages {64, 64, 9}, tm_kv4 half pages {64, 64, 4}.
 // F8 = true: FP8 cache; tm_kv9 loads a page's RoPE keys as one {64, 64} tile, tm_kv4 a half
 // page of raw codes {256, 64}; the codes of whole pages and the scales come by bulk copy.
-template <bool F8>
+template <bool F8, bool MM = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_constant__ CUtensorMap tm_kv4,
-                 const __grid_constant__ CUtensorMap tm_q9, const __grid_constant__ Params P) {
-    using L = Lay<F8>;
+                 const __grid_constant__ CUtensorMap tm_q9, const __grid_constant__ CUtensorMap tm_c8,
+                 const __grid_constant__ Params P) {
+    constexpr bool QF8 = F8 && MM;  // content scores on the FP8 tensor core
+    using L = Lay<F8, MM>;
     constexpr int KVS = L::kv_stages;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_u32(smem_raw);
@@ -505,6 +539,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
     };
     // Drain waits ignore the abort flag: they wait for hardware that is already running.
     volatile uint32_t *never = &ctrl->never;
+    Q8Extra *q8 = reinterpret_cast<Q8Extra *>(smem_raw + (data_s - raw_s) + L::q8_off);  // QF8 only
 
     if (rank == 0) {
         // ===================================== QK CTA =====================================
@@ -550,6 +585,21 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 st.adv(KVS);
                 return true;
             };
+            // FP8 with the content scores on the tensor core: codes (4 swizzled blocks), scales and
+            // RoPE keys straight into the page stage.
+            auto load_mm = [&](int blk) -> bool {
+                if (!wait(bar(ctrl->kv_empty[st.i]), st.ph ^ 1u, abort_flag)) return false;
+                const uint32_t dst = data_s + st.i * KV_STAGE;
+                mbar_arrive_expect_tx(bar(ctrl->kv_full[st.i]), 5 * CB + PG * 4);
+                tma_load_3d(dst, &tm_c8, 0, blk * PG, 0, bar(ctrl->kv_full[st.i]));
+                tma_load_2d(dst + (NCB - 1) * CB, &tm_kv9, 0, blk * PG, bar(ctrl->kv_full[st.i]));
+                bulk_load(dst + MM_SCALE_OFF, P.kv_scale + (size_t)blk * PG, PG * 4, bar(ctrl->kv_full[st.i]));
+                issued[st.i] = 1;
+                nph[st.i] = st.ph;
+                st.adv(KVS);
+                return true;
+            };
+            if (QF8) prefetch_tensormap(&tm_c8);
             while (ok && !it.done()) {
                 if (it.first) {
                     if (!(ok = load(&tm_q9, it.r * NH) && load(&tm_q9, it.r * NH + 64))) break;
@@ -560,7 +610,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 // timed-out wait: abort flags in both CTAs, error word, bounded drains, exit.
                 if (P.test_give_up && u == 1 && !(ok = wait(bar(ctrl->never_done), 0u, abort_flag, 20000ull)))
                     break;
-                if (!(ok = F8 ? load_f8(blk) : load(&tm_kv9, blk * PG))) break;
+                if (!(ok = QF8 ? load_mm(blk) : (F8 ? load_f8(blk) : load(&tm_kv9, blk * PG)))) break;
                 ++u;
                 it.next(P);
             }
@@ -607,12 +657,33 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 }
                 const uint32_t d = tmem + S_COL + sb.i * PG;
                 const uint32_t kvb = data_s + st.i * KV_STAGE;
+                if (QF8) {
+                    // e4m3 content: thread 0 the query's high part, thread 1 its low part (TMEM
+                    // columns Q_COL and Q_COL + 128: 4 codes per column, 8 columns per K = 32),
+                    // then thread 1 the RoPE part in bf16 (TMEM Q_COL + 256, the stage's block 8)
+                    constexpr uint32_t idesc8 = idesc_e4m3(128, PG);
+                    const uint32_t qa = tmem + Q_COL + (part ? 128u : 0u);
 #pragma unroll 1
-                for (int cb = cb0; cb < cb1; ++cb) {
+                    for (int kb = 0; kb < 4; ++kb) {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        mma_ts(d, tmem + Q_COL + (cb * 4 + k) * 8, sdesc_sw128(kvb + cb * CB + k * 32, 16, 1024),
-                               idesc, 1u);
+                        for (int k = 0; k < 4; ++k)
+                            mma_ts_f8(d, qa + (kb * 4 + k) * 8, sdesc_sw128(kvb + kb * CB + k * 32, 16, 1024), idesc8,
+                                      1u);
+                    }
+                    if (part) {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            mma_ts(d, tmem + Q_COL + 256 + k * 8,
+                                   sdesc_sw128(kvb + (NCB - 1) * CB + k * 32, 16, 1024), idesc, 1u);
+                    }
+                } else {
+#pragma unroll 1
+                    for (int cb = cb0; cb < cb1; ++cb) {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            mma_ts(d, tmem + Q_COL + (cb * 4 + k) * 8, sdesc_sw128(kvb + cb * CB + k * 32, 16, 1024),
+                                   idesc, 1u);
+                    }
                 }
                 if (!part) {
                     tc_fence_before();
@@ -657,8 +728,72 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 const int rr = h & 63;
                 const uint32_t rowa = data_s + ((h >> 6) ? q1.i : q0.i) * KV_STAGE + rr * 128;
                 const int cb0 = half ? 5 : 0, cb1 = half ? NCB : 5;
+                if (QF8) {
+                    // e4m3 query, per head: alpha = max|q_lat| / 448 (both halves' columns),
+                    // hi = e4m3(q / alpha), lo = e4m3(q / alpha - hi), so q ~ alpha (hi + lo) with
+                    // about 7 significant bits.  Codes into TMEM (4 per column): hi at Q_COL + c / 4,
+                    // lo at Q_COL + 128 + c / 4; the RoPE part as bf16(q_rope / alpha) at Q_COL + 256.
+                    const int ce = half ? NCB - 1 : 5;  // content blocks of this half: [cb0, ce)
+                    float am = 0.f;
 #pragma unroll 1
-                for (int cb = cb0; cb < cb1; ++cb) {
+                    for (int cb = cb0; cb < ce; ++cb)
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const uint4 x = ld_shared_v4(rowa + cb * CB + ((c ^ (rr & 7)) << 4));
+                            const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 f = bf16x2_to_float2(xw[e]);
+                                am = fmaxf(am, fmaxf(fabsf(f.x), fabsf(f.y)));
+                            }
+                        }
+                    q8->qamax[half][h] = am;
+                    named_sync(BAR_Q, SM_THREADS);
+                    const float alpha = fmaxf(fmaxf(q8->qamax[0][h], q8->qamax[1][h]) / 448.f, FLT_MIN);
+                    const float ia = 1.f / alpha;
+                    if (!half) q8->qalpha[h] = alpha;
+#pragma unroll 1
+                    for (int cb = cb0; cb < ce; ++cb) {
+                        uint32_t hw[16], lw[16];
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const uint4 x = ld_shared_v4(rowa + cb * CB + ((c ^ (rr & 7)) << 4));
+                            const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+                            uint32_t hc[4], lc[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 f = bf16x2_to_float2(xw[e]);
+                                const float y0 = f.x * ia, y1 = f.y * ia;
+                                const uint32_t h2 = f32x2_to_e4m3x2(y0, y1);
+                                const float2 b = e4m3x2_to_float2(h2);
+                                hc[e] = h2;
+                                lc[e] = f32x2_to_e4m3x2(y0 - b.x, y1 - b.y);
+                            }
+                            hw[2 * c] = hc[0] | (hc[1] << 16);
+                            hw[2 * c + 1] = hc[2] | (hc[3] << 16);
+                            lw[2 * c] = lc[0] | (lc[1] << 16);
+                            lw[2 * c + 1] = lc[2] | (lc[3] << 16);
+                        }
+                        tmem_st16(tmem + lane_base + Q_COL + cb * 16, hw);
+                        tmem_st16(tmem + lane_base + Q_COL + 128 + cb * 16, lw);
+                    }
+                    if (half) {  // the RoPE part
+                        uint32_t v[32];
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const uint4 x = ld_shared_v4(rowa + (NCB - 1) * CB + ((c ^ (rr & 7)) << 4));
+                            const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 f = bf16x2_to_float2(xw[e]);
+                                v[4 * c + e] = pack_bf16x2(f.x * ia, f.y * ia);
+                            }
+                        }
+                        tmem_st32(tmem + lane_base + Q_COL + 256, v);
+                    }
+                }
+#pragma unroll 1
+                for (int cb = cb0; cb < (QF8 ? cb0 : cb1); ++cb) {
                     uint32_t v[32];
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
@@ -688,7 +823,38 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
             // Pages are converted one ahead of the softmax: the next page of the segment before
             // this page's softmax, a segment's first page right after its Q copy.
             Ring cg{0, 0};
+            int uc = 0;  // FP8 tensor-core QK: pages prepared so far (index of the scale ring)
             auto convert = [&](Ring c) -> bool {
+                if (QF8) {
+                    // The page's RoPE keys divided by the token's scale (in place, 16 values per
+                    // thread), so that S = alpha_h s_j (hi + lo).c8_j + (q_rope / alpha_h).(k_j / s_j)
+                    // needs one per-column factor; the factors go to the scale ring for the softmax.
+                    const bool w = wait(bar(ctrl->kv_full[c.i]), c.ph, abort_flag);
+                    if (named_red_or(!w, BAR_CONV, SM_THREADS)) return false;
+                    const uint32_t stage = data_s + c.i * KV_STAGE;
+                    const float *scl = reinterpret_cast<const float *>(smem_raw + (stage - raw_s) + MM_SCALE_OFF);
+#pragma unroll
+                    for (int q = t; q < PG * 8; q += SM_THREADS) {  // 512 chunks of 8 keys
+                        const int j = q >> 3, cc = q & 7;
+                        const uint32_t a = stage + (NCB - 1) * CB + j * 128 + ((cc ^ (j & 7)) << 4);
+                        const uint4 x = ld_shared_v4(a);
+                        const float inv = 1.f / scl[j];
+                        const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+                        uint32_t o[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = bf16x2_to_float2(xw[e]);
+                            o[e] = pack_bf16x2(f.x * inv, f.y * inv);
+                        }
+                        st_shared_v4(a, o[0], o[1], o[2], o[3]);
+                    }
+                    if (t < PG) q8->pscale[uc % 3][t] = scl[t] * P.scale_log2;
+                    ++uc;
+                    fence_proxy_async_smem();
+                    named_sync(BAR_CONV, SM_THREADS);  // the factors are visible to every softmax thread
+                    if (lane == 0) mbar_arrive(bar(ctrl->conv_full[c.i]));
+                    return true;
+                }
                 const bool w = wait(bar(ctrl->stg_full[cg.i]), cg.ph, abort_flag) &&
                                wait(bar(ctrl->kv_empty[c.i]), c.ph ^ 1u, abort_flag);
                 if (named_red_or(!w, BAR_CONV, SM_THREADS)) return false;
@@ -748,6 +914,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 const int valid = it.valid();
                 const int r = it.r;
                 // ---- online softmax (log2 units; scale folded into one FFMA) ----
+                float sl2 = P.scale_log2;
+                if (QF8) {  // per-column factors alpha_h s_j log2(e)/sqrt(d): scale first, then one
+                    const float al = q8->qalpha[h];
+                    const float *ps = q8->pscale[u % 3];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        mine[j] *= al * ps[half * 32 + j];
+                        other[j] *= al * ps[(half ^ 1) * 32 + j];
+                    }
+                    sl2 = 1.f;
+                }
                 if (valid < PG) {
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
@@ -755,7 +932,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                         if ((half ^ 1) * 32 + j >= valid) other[j] = -INFINITY;
                     }
                 }
-                const float mx = fmaxf(max32(mine), max32(other)) * P.scale_log2;
+                const float mx = fmaxf(max32(mine), max32(other)) * sl2;
                 float m_new = m_used, fac = 1.f;
                 if (first) {
                     m_new = mx;
@@ -768,8 +945,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kv9, const __grid_consta
                 uint32_t pk[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const float p0 = fast_exp2(fmaf(mine[2 * j], P.scale_log2, -m_new));
-                    const float p1 = fast_exp2(fmaf(mine[2 * j + 1], P.scale_log2, -m_new));
+                    const float p0 = fast_exp2(fmaf(mine[2 * j], sl2, -m_new));
+                    const float p1 = fast_exp2(fmaf(mine[2 * j + 1], sl2, -m_new));
                     s0 += p0;
                     s1 += p1;
                     pk[j] = pack_bf16x2(p0, p1);
@@ -1196,19 +1373,21 @@ combine_tc_kernel(const int32_t *__restrict__ seg_range, const uint32_t *__restr
 }
 
 // ---- host side ------------------------------------------------------------------------------
-int g_pairs[2][64] = {};
+int g_pairs[3][64] = {};  // [bf16 | FP8 | FP8 with the content scores on the FP8 tensor core][device]
 std::mutex g_pairs_mu;
 
 // Co-resident clusters of the kernel on the current device (cached per device; the first call
 // on a device sets the kernel's shared-memory attribute and queries the occupancy, under a lock
 // so that concurrent first calls from several host threads do it once).
-template <bool F8>
+template <bool F8, bool MM = false>
 int tc_pairs() {
+    constexpr int K = F8 ? (MM ? 2 : 1) : 0;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
     std::lock_guard<std::mutex> lk(g_pairs_mu);
-    if (g_pairs[F8][dev]) return g_pairs[F8][dev];
-    if (cudaFuncSetAttribute(decode_tc_kernel<F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay<F8>::smem) !=
+    if (g_pairs[K][dev]) return g_pairs[K][dev];
+    if (cudaFuncSetAttribute(decode_tc_kernel<F8, MM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Lay<F8, MM>::smem) !=
         cudaSuccess)
         return 0;
     int sms = 148;
@@ -1216,7 +1395,7 @@ int tc_pairs() {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (sms / 2));
     cfg.blockDim = dim3(THREADS);
-    cfg.dynamicSmemBytes = Lay<F8>::smem;
+    cfg.dynamicSmemBytes = Lay<F8, MM>::smem;
     cudaLaunchAttribute attr;
     attr.id = cudaLaunchAttributeClusterDimension;
     attr.val.clusterDim.x = 2;
@@ -1225,15 +1404,16 @@ int tc_pairs() {
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, decode_tc_kernel<F8>, &cfg) != cudaSuccess || n < 1) {
+    if (cudaOccupancyMaxActiveClusters(&n, decode_tc_kernel<F8, MM>, &cfg) != cudaSuccess || n < 1) {
         cudaGetLastError();
         n = sms / 2;
     }
-    g_pairs[F8][dev] = n;
+    g_pairs[K][dev] = n;
     return n;
 }
 int tc_pairs(const mla_dims_t &d) {
-    return d.kv_dtype == MLA_DTYPE_FP8_E4M3 ? tc_pairs<true>() : tc_pairs<false>();
+    if (d.kv_dtype != MLA_DTYPE_FP8_E4M3) return tc_pairs<false>();
+    return (d.flags & MLA_FLAG_FP8_MMA) ? tc_pairs<true, true>() : tc_pairs<true>();
 }
 
 struct TcWs {
@@ -1287,7 +1467,8 @@ cudaError_t launch_decode_tc(const mla_dims_t &d, int B, int s_q, const void *q_
     if (pairs < 1) return cudaErrorNotSupported;
     TcWs w;
     if (tc_layout(pairs, rows, reinterpret_cast<char *>(ws), &w) > ws_bytes) return cudaErrorInvalidValue;
-    CUtensorMap tm_kv9, tm_kv4, tm_q9;
+    CUtensorMap tm_kv9, tm_kv4, tm_q9, tm_c8;
+    const bool mm = f8 && (d.flags & MLA_FLAG_FP8_MMA);
     const uint64_t pool_rows = (uint64_t)num_blocks * PG, q_rows = (uint64_t)rows * NH;
     const bool maps =
         f8 ? (tmap_bf16_2d(&tm_kv9, kr_pool, ROW - DC, pool_rows, (ROW - DC) * 2, 64, PG) &&
@@ -1295,6 +1476,10 @@ cudaError_t launch_decode_tc(const mla_dims_t &d, int B, int s_q, const void *q_
            : (tmap_bf16_colblocks(&tm_kv9, kv_pool, pool_rows, ROW, ROW * 2, PG, NCB) &&
               tmap_bf16_colblocks(&tm_kv4, kv_pool, pool_rows, ROW, ROW * 2, PG, 4));
     if (!maps || !tmap_bf16_colblocks(&tm_q9, q_abs, q_rows, ROW, ROW * 2, 64, NCB)) return cudaErrorInvalidValue;
+    // FP8 with the content scores on the tensor core: the codes as 4 K-major 128-byte blocks
+    // per page (the map is passed, unused, to the other instantiations)
+    if (mm ? !tmap_u8_colblocks(&tm_c8, kv_pool, pool_rows, DC, DC, PG, 4) : false) return cudaErrorInvalidValue;
+    if (!mm) tm_c8 = tm_q9;
     unsigned *err = device_error_word();
     cudaError_t e;
     Params P;
@@ -1324,7 +1509,7 @@ cudaError_t launch_decode_tc(const mla_dims_t &d, int B, int s_q, const void *q_
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs);
     cfg.blockDim = dim3(THREADS);
-    cfg.dynamicSmemBytes = f8 ? Lay<true>::smem : Lay<false>::smem;
+    cfg.dynamicSmemBytes = mm ? Lay<true, true>::smem : (f8 ? Lay<true>::smem : Lay<false>::smem);
     cfg.stream = st;
     cfg.attrs = &pdl;
 #ifdef MLA_NO_PDL
@@ -1332,8 +1517,9 @@ cudaError_t launch_decode_tc(const mla_dims_t &d, int B, int s_q, const void *q_
 #else
     cfg.numAttrs = 1;
 #endif
-    e = f8 ? cudaLaunchKernelEx(&cfg, decode_tc_kernel<true>, tm_kv9, tm_kv4, tm_q9, P)
-           : cudaLaunchKernelEx(&cfg, decode_tc_kernel<false>, tm_kv9, tm_kv4, tm_q9, P);
+    e = mm   ? cudaLaunchKernelEx(&cfg, decode_tc_kernel<true, true>, tm_kv9, tm_kv4, tm_q9, tm_c8, P)
+        : f8 ? cudaLaunchKernelEx(&cfg, decode_tc_kernel<true>, tm_kv9, tm_kv4, tm_q9, tm_c8, P)
+             : cudaLaunchKernelEx(&cfg, decode_tc_kernel<false>, tm_kv9, tm_kv4, tm_q9, tm_c8, P);
     if (e != cudaSuccess) return e;
     if (fuse)
         return launch_combine_out_proj_tc(d, rows, w.seg_range, w.o, w.m, w.l, o_lat, lse, fuse->w_uv, fuse->o,

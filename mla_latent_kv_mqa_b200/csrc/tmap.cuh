@@ -64,6 +64,22 @@ inline bool tmap_u8_rows(CUtensorMap *m, const void *base, uint64_t inner, uint6
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+// 3-D byte "column-block" map over rows of `cols` bytes (`row_bytes` apart): coordinates
+// (x in a 128-byte column block, row, column block); a box {128, box_rows, nblk} lands as nblk
+// consecutive [box_rows x 128 B] tiles with 128-byte swizzle (the K-major layout of 8-bit
+// tensor-core operands).
+inline bool tmap_u8_colblocks(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint64_t row_bytes,
+                              uint32_t box_rows, uint32_t nblk) {
+    auto fn = tmap_encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[3] = {128, (cuuint64_t)rows, (cuuint64_t)(cols / 128)};
+    cuuint64_t gstride[2] = {(cuuint64_t)row_bytes, 128};
+    cuuint32_t box[3] = {128, box_rows, nblk};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), gdim, gstride, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 inline bool tmap_bf16_2d(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t row_bytes,
                          uint32_t box_inner, uint32_t box_rows) {
     return tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, inner, rows, row_bytes, box_inner, box_rows);

@@ -38,6 +38,7 @@ MLA_DTYPE_FP8_E4M3 = 2
 MLA_FLAG_SIMT_DECODE = 1
 MLA_FLAG_SIMT_PROJ = 2
 MLA_FLAG_TEST_GIVE_UP = 4
+MLA_FLAG_FP8_MMA = 8
 
 
 class MLAError(RuntimeError):

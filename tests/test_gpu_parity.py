@@ -240,3 +240,37 @@ def test_workspace_contents_do_not_matter(fill):
     got = run.step()
     for x, y in zip(ref[1:], got[1:]):
         assert torch.equal(x, y)
+
+
+# ---------------------------------------------------------------------------------------------
+# FP8 cache with the content scores on the FP8 tensor core (MLA_FLAG_FP8_MMA): the same
+# bounds as the FP8 cache (relative L2 <= 3e-2 against the oracle on its own dequantised cache)
+# ---------------------------------------------------------------------------------------------
+
+FP8_MMA = {
+    "fp8_mma_sq2": dict(seed=41, seq_lens=[300, 2, 65, 128], s_q=2, kv_dtype="fp8"),
+    "fp8_mma_ragged_permuted": dict(seed=42, seq_lens=[200, 64, 1, 129, 700], kv_dtype="fp8", permute=True,
+                                    spare=4),
+    "fp8_mma_lognormal": dict(seed=43, seq_lens=[2000], lognormal_tokens=True, kv_dtype="fp8"),
+    "fp8_mma_long_rows": dict(seed=44, seq_lens=[5000, 3000], s_q=2, kv_dtype="fp8"),
+}
+
+
+@pytest.mark.parametrize("case", sorted(FP8_MMA))
+def test_fp8_tensor_core_scores_match_oracle(oracle_mod, case):
+    import mla_latent_kv_mqa_b200.native as Nat
+    wl = W.make_decode(name=case, **FP8_MMA[case])
+    run = GpuRun(wl, flags=Nat.MLA_FLAG_FP8_MMA)
+    run.fill_cache()
+    got = run.step()
+    assert Nat.mla_get_last_device_error() == 0
+    rows, heads, ref = oracle_ref(wl, oracle_mod)
+    e = _check(wl, got, ref, rows, heads, FP8_REL, None)
+    # and against the default FP8 path (bf16 dequantisation) on the same cache
+    run2 = GpuRun(wl)
+    run2.fill_cache()
+    got2 = run2.step()
+    assert rel_l2(got[1].cpu().numpy(), got2[1].cpu().numpy()) <= FP8_REL, e
+    # bitwise reproducible
+    again = run.step()
+    assert torch.equal(again[1], got[1]) and torch.equal(again[2], got[2])
