@@ -191,8 +191,11 @@ prefill_kv_up_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_cons
                 mma_ss(tmem, sdesc_sw128(a + k * 32, 16, 1024), sdesc_sw128(b + k * 32, 16, 1024), idesc,
                        (kc | k) != 0 ? 1u : 0u);
             mma_commit(bar(ctrl->empty[s]));
-            if (issued < PDC / 64) {
-                if (!(ok = wait(bar(ctrl->empty[s]), (kc / UP_STAGES) & 1u, abort_flag))) break;
+            // refill the stage of the previous chunk (its MMAs are queued before this chunk's, so
+            // waiting for them keeps this chunk's MMAs in the tensor pipe meanwhile)
+            if (kc >= 1 && issued < PDC / 64) {
+                const int ps = (kc - 1) % UP_STAGES;
+                if (!(ok = wait(bar(ctrl->empty[ps]), ((kc - 1) / UP_STAGES) & 1u, abort_flag))) break;
                 load(issued++);
             }
         }
@@ -252,7 +255,8 @@ prefill_kv_up_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_cons
 // CTA = (query tile qt, head h, prompt b), 320 threads: warp 0 loads (TMA; lane 0 Q and K,
 // lane 1 V), warp 1 issues the MMAs, warps 2-9 run the softmax, two warps per TMEM lane
 // quarter (warp w reads lanes 32 (w % 4) ...), each on 64 of the tile's 128 keys; the two
-// exchange their row maxima through shared memory once per tile.
+// exchange their row maxima through shared memory once per tile.  (Reading the whole row in
+// both warps instead, to skip the exchange, measured slower.)
 // Shared: Q [3 blocks x 128 rows x 128 B] 48 KB; K ring 2 x (Kh 2 blocks + kr 1 block) 48 KB;
 // V ring 2 x (2 blocks of [128 keys x 64 d]) 32 KB.  TMEM: S0 [0,128), S1 [128,256), O [256,384).
 // Pipeline (MMA issue order): QK0, QK1, PV0, QK2, PV1, QK3, ...; P_j overwrites S_j's first 64
@@ -264,20 +268,22 @@ constexpr int AT_KS = 3 * AT_QB;                // K stage: 48 KB
 constexpr int AT_V = AT_K + 2 * AT_KS;          // 144 KB
 constexpr int AT_VS = 2 * AT_QB;                // V stage: 32 KB
 constexpr int AT_DATA = AT_V + 2 * AT_VS;       // 208 KB
-constexpr int AT_SMEM = 1024 + AT_DATA + 4096;
+constexpr int AT_SMEM = 1024 + AT_DATA + 5120;
 constexpr int AT_THREADS = 320;
-constexpr uint32_t S_COL0 = 0, O_COL = 256;
+constexpr int NSB = 3;                             // S buffers in TMEM
+constexpr uint32_t S_COL0 = 0, O_COL = NSB * 128;  // S: [0, 384), O: [384, 512)
 constexpr float kRescaleLog2 = 8.f;  // O is rescaled only when the running max grows by > 2^8
 
 struct __align__(8) AtCtrl {
-    uint64_t q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_ready[2], pv_done[2], idle;
-    uint64_t xbar[4][2];      // the two softmax warps of a lane quarter meet here (per S buffer)
+    uint64_t q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[NSB], p_ready[NSB], pv_done[NSB], idle;
+    uint64_t xbar[4][1 + NSB];  // the two softmax warps of a lane quarter meet here: [0] the final row
+                                // sums, [1 + s] the row maxima of S buffer s
+    float xmax[NSB][2][128];  // [S buffer][half][row]: row max of each half's raw scores
     uint32_t tmem_base, abort;
     uint32_t never;           // stays 0: the abort word of drain waits
-    float xmax[2][2][128];    // [S buffer][half][row]: row max of each half's raw scores
     float xsum[2][128];       // [half][row]: the final row sums
 };
-static_assert(sizeof(AtCtrl) <= 4096, "control block");
+static_assert(sizeof(AtCtrl) <= 5120, "control block");
 
 __global__ void __launch_bounds__(AT_THREADS, 1)
 prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -311,13 +317,15 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mbar_init(bar(ctrl->k_empty[i]), 1);
             mbar_init(bar(ctrl->v_full[i]), 1);
             mbar_init(bar(ctrl->v_empty[i]), 1);
+        }
+        for (int i = 0; i < NSB; ++i) {
             mbar_init(bar(ctrl->s_full[i]), 1);
             mbar_init(bar(ctrl->p_ready[i]), 8);
             mbar_init(bar(ctrl->pv_done[i]), 1);
         }
         mbar_init(bar(ctrl->idle), 1);
         for (int qq = 0; qq < 4; ++qq)
-            for (int i = 0; i < 2; ++i) mbar_init(bar(ctrl->xbar[qq][i]), 2);
+            for (int i = 0; i < 1 + NSB; ++i) mbar_init(bar(ctrl->xbar[qq][i]), 2);
         ctrl->abort = 0;
         ctrl->never = 0;
         fence_mbarrier_init_cluster();
@@ -373,10 +381,10 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             constexpr uint32_t idesc_pv = idesc_bf16(128, 128, false, true);
             bool ok = wait(bar(ctrl->q_full), 0u, abort_flag);
             auto qk = [&](int j) {
-                const int s = j & 1;
+                const int s = j & 1;  // K stage; S buffer j % NSB
                 if (!wait(bar(ctrl->k_full[s]), (uint32_t)(j >> 1) & 1u, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t kb = data_s + AT_K + s * AT_KS, d = tmem + S_COL0 + s * 128;
+                const uint32_t kb = data_s + AT_K + s * AT_KS, d = tmem + S_COL0 + (j % NSB) * 128;
 #pragma unroll
                 for (int cb = 0; cb < 3; ++cb)
 #pragma unroll
@@ -384,25 +392,23 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         mma_ss(d, sdesc_sw128(data_s + AT_Q + cb * AT_QB + k * 32, 16, 1024),
                                sdesc_sw128(kb + cb * AT_QB + k * 32, 16, 1024), idesc_qk, (cb | k) != 0 ? 1u : 0u);
                 mma_commit(bar(ctrl->k_empty[s]));
-                mma_commit(bar(ctrl->s_full[s]));
+                mma_commit(bar(ctrl->s_full[j % NSB]));
                 return true;
             };
-            if (ok) ok = qk(0);
-            if (ok && n_kt > 1) ok = qk(1);
+            for (int j = 0; ok && j < NSB && j < n_kt; ++j) ok = qk(j);
             for (int j = 0; ok && j < n_kt; ++j) {
-                const int s = j & 1;
-                const uint32_t ph = (uint32_t)(j >> 1) & 1u;
-                if (!(ok = wait(bar(ctrl->p_ready[s]), ph, abort_flag))) break;
-                if (!(ok = wait(bar(ctrl->v_full[s]), ph, abort_flag))) break;
+                const int s = j & 1, sb = j % NSB;
+                if (!(ok = wait(bar(ctrl->p_ready[sb]), (uint32_t)(j / NSB) & 1u, abort_flag))) break;
+                if (!(ok = wait(bar(ctrl->v_full[s]), (uint32_t)(j >> 1) & 1u, abort_flag))) break;
                 tc_fence_after();
-                const uint32_t vb = data_s + AT_V + s * AT_VS, p = tmem + S_COL0 + s * 128;
+                const uint32_t vb = data_s + AT_V + s * AT_VS, p = tmem + S_COL0 + sb * 128;
 #pragma unroll
                 for (int kk = 0; kk < PT / 16; ++kk)
                     mma_ts(tmem + O_COL, p + kk * 8, sdesc_sw128(vb + kk * 2048, AT_QB, 1024), idesc_pv,
                            (j | kk) != 0 ? 1u : 0u);
                 mma_commit(bar(ctrl->v_empty[s]));
-                mma_commit(bar(ctrl->pv_done[s]));
-                if (j + 2 < n_kt) ok = qk(j + 2);
+                mma_commit(bar(ctrl->pv_done[sb]));
+                if (j + NSB < n_kt) ok = qk(j + NSB);
             }
             if (!ok) *abort_flag = 1;
             // no MMA may still run when TMEM is released
@@ -420,8 +426,8 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         bool ok = true;
         int j = 0;
         for (; j < n_kt; ++j) {
-            const int s = j & 1;
-            const uint32_t ph = (uint32_t)(j >> 1) & 1u;
+            const int s = j % NSB;
+            const uint32_t ph = (uint32_t)(j / NSB) & 1u;
             if (!(ok = __all_sync(0xffffffffu, wait(bar(ctrl->s_full[s]), ph, abort_flag)))) break;
             tc_fence_after();
             uint32_t v[64];
@@ -430,23 +436,24 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tmem_wait_ld();
             // keys j*128 + cbase + c with c <= lim are visible (causal, and inside the prompt)
             const int lim = min(qi, L - 1) - j * PT - cbase;
-            float pm = -INFINITY;  // row max of this warp's raw scores
+            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // row max of this warp's raw scores
             if (__all_sync(0xffffffffu, lim >= 63)) {
 #pragma unroll
-                for (int c = 0; c < 64; ++c) pm = fmaxf(pm, __uint_as_float(v[c]));
+                for (int c = 0; c < 64; ++c) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(v[c]));
             } else {
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
                     const float x = c <= lim ? __uint_as_float(v[c]) : -INFINITY;
                     v[c] = __float_as_uint(x);
-                    pm = fmaxf(pm, x);
+                    mx[c & 3] = fmaxf(mx[c & 3], x);
                 }
             }
+            const float pm = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             // the row max over both halves: exchange with the partner warp of this quarter
             ctrl->xmax[s][half][row] = pm;
             __syncwarp();
-            if (lane == 0) mbar_arrive(xbar0 + s * 8);
-            if (!(ok = __all_sync(0xffffffffu, wait(xbar0 + s * 8, ph, abort_flag)))) break;
+            if (lane == 0) mbar_arrive(xbar0 + (1 + s) * 8);
+            if (!(ok = __all_sync(0xffffffffu, wait(xbar0 + (1 + s) * 8, ph, abort_flag)))) break;
             const float mt = fmaxf(pm, ctrl->xmax[s][half ^ 1][row]) * scale_log2;
             float fac = 1.f;
             if (mt > m_run + kRescaleLog2) {  // also the first visible key (m_run = -inf)
@@ -458,7 +465,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // half of the 128 value columns)
             if (j > 0 && __any_sync(0xffffffffu, fac != 1.f)) {
                 const int pj = j - 1;
-                if (!(ok = __all_sync(0xffffffffu, wait(bar(ctrl->pv_done[pj & 1]), (uint32_t)(pj >> 1) & 1u,
+                if (!(ok = __all_sync(0xffffffffu, wait(bar(ctrl->pv_done[pj % NSB]), (uint32_t)(pj / NSB) & 1u,
                                                         abort_flag))))
                     break;
                 tc_fence_after();
@@ -475,16 +482,16 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             const bool live = m_run != -INFINITY;
             const float nm = -m_run;
-            float sum = 0.f;
+            float sum[4] = {0.f, 0.f, 0.f, 0.f};
             uint32_t pk[32];
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
                 const float p0 = live ? ex2(fmaf(__uint_as_float(v[2 * c]), scale_log2, nm)) : 0.f;
                 const float p1 = live ? ex2(fmaf(__uint_as_float(v[2 * c + 1]), scale_log2, nm)) : 0.f;
-                sum += p0 + p1;
+                sum[c & 3] += p0 + p1;
                 pk[c] = pack_bf16x2(p0, p1);
             }
-            l_run += sum;
+            l_run += (sum[0] + sum[1]) + (sum[2] + sum[3]);
             // P over the first 64 columns of this S buffer: keys 2c, 2c+1 in column c
             tmem_st32(lane_base + S_COL0 + s * 128 + half * 32, pk);
             tmem_wait_st();
@@ -494,14 +501,13 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         if (ok) {
             const int lj = n_kt - 1;
-            ok = __all_sync(0xffffffffu, wait(bar(ctrl->pv_done[lj & 1]), (uint32_t)(lj >> 1) & 1u, abort_flag));
+            ok = __all_sync(0xffffffffu, wait(bar(ctrl->pv_done[lj % NSB]), (uint32_t)(lj / NSB) & 1u, abort_flag));
         }
         if (ok) {  // the row sum over both halves (one more exchange, tile index n_kt)
-            const int s = n_kt & 1;
             ctrl->xsum[half][row] = l_run;
             __syncwarp();
-            if (lane == 0) mbar_arrive(xbar0 + s * 8);
-            ok = __all_sync(0xffffffffu, wait(xbar0 + s * 8, (uint32_t)(n_kt >> 1) & 1u, abort_flag));
+            if (lane == 0) mbar_arrive(xbar0);  // the barrier's only use: phase 0
+            ok = __all_sync(0xffffffffu, wait(xbar0, 0u, abort_flag));
         }
         if (ok) {
             tc_fence_after();
