@@ -2,10 +2,12 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference] [--config v3]
 
-A step is the whole decode path over one batch: mla_cache_append (the batch's new tokens),
-mla_absorb_q, mla_decode (split-KV attention, scheduled in its prologue, + log-sum-exp combine) and
-mla_out_proj.  The default workload is the DeepSeek-V3-shaped single-layer decode (n_h=128,
-d_h=128, d_c=512, d_R=64, bf16 cache, batch 16, context 4096, s_q=1, 64-token pages).
+A step is the whole decode path over one batch: mla_append_absorb (the batch's new tokens into
+the cache and the absorbed queries, one launch), mla_decode (split-KV attention, scheduled in
+its prologue, + log-sum-exp combine) and mla_out_proj (o in the activation dtype).  The default
+workload is the DeepSeek-V3-shaped single-layer decode (n_h=128, d_h=128, d_c=512, d_R=64, bf16
+cache, batch 16, context 4096, s_q=1, 64-token pages).  The same line carries the other
+workloads and the MHA-mode prefill (mla_prefill) under "configs".
 
 Timing: CUDA events on the launching stream around each step, after W warm-up steps; the L2
 is flushed (a 512 MiB write) before every timed step, outside the events.  Under torchrun
