@@ -442,6 +442,69 @@ def prefill_flops(wl):
     return attn, up
 
 
+SEQSPLIT = ("long workload (V3 dims, 4 x 131072 tokens, log-normal norms) split over 2 ranks by pages, one rank "
+            "emulated on one GPU: its mla_decode over half of every sequence's pages, then mla_lse_merge_prepare and "
+            "mla_lse_merge_finish (the two all-reduces between them are not in the time)")
+
+
+def measure_seqsplit(K, warmup, dev, world_emul=2):
+    """K timed rank-0 steps of the sequence split (CUDA graph, L2 flushed before each)."""
+    import torch
+    from mla_latent_kv_mqa_b200 import native as N
+    from mla_latent_kv_mqa_b200 import seqsplit as S
+    from tests.harness import GpuRun
+    wl = make_workload("long")
+    run = GpuRun(wl, dev=dev)
+    run.fill_cache()
+    d = run.dims
+    bounds = S.page_bounds(wl.seq_lens, world_emul, wl.dims.page)
+    _, n = S.token_ranges(wl.seq_lens, bounds, 0, wl.dims.page)
+    bt = torch.from_numpy(S.local_block_table(wl.block_table, bounds, 0)).to(dev)
+    lens = torch.from_numpy(n.astype(np.int32)).to(dev)
+    rows = wl.T
+    q_abs = run.layer.absorb(run.q_c, run.q_r, run.q_pos)
+    o_lat = torch.empty((rows, d.n_h, d.d_c), dtype=torch.float32, device=dev)
+    lse = torch.empty((rows, d.n_h), dtype=torch.float32, device=dev)
+    lse_max = torch.empty_like(lse)
+    acc = torch.empty(rows * d.n_h * (d.d_c + 1), dtype=torch.float32, device=dev)
+    out = torch.empty_like(o_lat)
+    out_lse = torch.empty_like(lse)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        run.layer.decode(run.cache, q_abs, bt, lens, 1, int(n.max()), o_lat=o_lat, lse=lse)
+        lse_max.copy_(lse)  # stands in for the all-reduce(max)
+        N.mla_lse_merge_prepare(rows, d.n_h, d.d_c, o_lat, lse, lse_max, acc, stream)
+        N.mla_lse_merge_finish(rows, d.n_h, d.d_c, acc, lse_max, out, out_lse, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(warmup, 3)):
+            flush.fill_(1)
+            step()
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        for k in range(K):
+            flush.fill_(k & 0xFF)
+            ev[k][0].record(stream)
+            g.replay()
+            ev[k][1].record(stream)
+        stream.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / K
+    if N.mla_get_last_device_error() != 0:
+        raise SystemExit("device error during the sequence-split measurement")
+    del g, run, flush
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return {"workload": SEQSPLIT, "ranks": world_emul, "steps": K, "rank_ms": ms,
+            "tokens_per_s_if_ranks_run_together": rows / (ms * 1e-3),
+            "exchange_bytes_per_allreduce": {"max": rows * d.n_h * 4, "sum": rows * d.n_h * (d.d_c + 1) * 4},
+            "gpu_launches": 5 * K}
+
+
 def measure_prefill(K, warmup, dev, with_clock=True, lens=None):
     """K timed mla_prefill calls (CUDA graph of the one call, L2 flushed before each)."""
     import torch
@@ -623,6 +686,7 @@ def run_mine(args):
         if not args.no_cpu_baseline:
             c["cpu_baseline"] = prefill_cpu_baseline(wlp)
         configs["prefill"] = c
+        configs["seqsplit"] = measure_seqsplit(k2, args.warmup, dev)
         del wlp
         line["configs"] = configs
     if rank == 0:
