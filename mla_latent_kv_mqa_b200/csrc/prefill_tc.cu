@@ -43,6 +43,71 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// ---- packed fp32 pairs (Blackwell f32x2 arithmetic: two lanes of work per instruction) ----
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+    return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
+}
+__device__ __forceinline__ float f2lo(uint64_t a) { return __uint_as_float((uint32_t)a); }
+__device__ __forceinline__ float f2hi(uint64_t a) { return __uint_as_float((uint32_t)(a >> 32)); }
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 2^x for a pair, on the FMA pipe instead of the MUFU unit (whose 16 results per clock per SM
+// otherwise bound the softmax).  Cody-Waite style: x = j + f with j = rint(x), taken by adding
+// 1.5 * 2^23 (j then sits in the low mantissa bits of t), f in [-1/2, 1/2]; 2^f by a degree-3
+// polynomial whose coefficients are the minimax fit of the relative error on [-1/2, 1/2]
+// (Remez exchange, rounded to fp32; max relative error 7.5e-5, 1/26 of the bf16 rounding that P
+// gets next); 2^j enters as j added to the exponent field.  x is clamped to >= -126 first, so
+// the result stays a non-negative finite number (2^-126 or less where x was lower).
+constexpr float kEx2C0 = 0.9999280571937561f, kEx2C1 = 0.6932609677314758f;
+constexpr float kEx2C2 = 0.2426111251115799f, kEx2C3 = 0.0551716685295105f;
+__device__ __forceinline__ uint64_t ex2_poly2(uint64_t x) {
+    constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+    x = f2pack(fmaxf(f2lo(x), -126.f), fmaxf(f2hi(x), -126.f));
+    const uint64_t t = add2(x, f2pack(kRound, kRound));
+    const uint64_t f = sub2(x, sub2(t, f2pack(kRound, kRound)));
+    uint64_t p = fma2(f2pack(kEx2C3, kEx2C3), f, f2pack(kEx2C2, kEx2C2));
+    p = fma2(p, f, f2pack(kEx2C1, kEx2C1));
+    p = fma2(p, f, f2pack(kEx2C0, kEx2C0));
+    const uint32_t lo = (uint32_t)p + ((uint32_t)t << 23), hi = (uint32_t)(p >> 32) + ((uint32_t)(t >> 32) << 23);
+    return (uint64_t)lo | ((uint64_t)hi << 32);
+}
+
+// P = 2^(S scale_log2 - m) for this warp's 64 keys of a row: packed bf16 pairs into pk, the fp32
+// sum returned.  With POLY, the pairs c with c % 4 == 3 take ex2_poly2 (a quarter of the
+// exponentials); only for tiles without masked keys, whose scores are all finite.
+template <bool POLY>
+__device__ __forceinline__ float softmax_exp(const uint32_t (&v)[64], float scale_log2, float nm, uint32_t (&pk)[32]) {
+    const uint64_t sl2 = f2pack(scale_log2, scale_log2), nm2 = f2pack(nm, nm);
+    uint64_t acc[2] = {0ull, 0ull};
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        const uint64_t x = fma2(f2pack(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])), sl2, nm2);
+        uint64_t p;
+        if (POLY && (c & 3) == 3)
+            p = ex2_poly2(x);
+        else
+            p = f2pack(ex2(f2lo(x)), ex2(f2hi(x)));
+        acc[c & 1] = add2(acc[c & 1], p);
+        pk[c] = pack_bf16x2(f2lo(p), f2hi(p));
+    }
+    const uint64_t a = add2(acc[0], acc[1]);
+    return f2lo(a) + f2hi(a);
+}
+
 __device__ __forceinline__ int seq_of(const int32_t *cu, int B, int t) {
     int lo = 0, hi = B;  // largest b with cu[b] <= t
     while (hi - lo > 1) {
@@ -252,15 +317,16 @@ prefill_kv_up_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_cons
 }
 
 // ---- 3. causal attention ------------------------------------------------------------------
-// CTA = (query tile qt, head h, prompt b), 320 threads: warp 0 loads (TMA; lane 0 Q and K,
-// lane 1 V), warp 1 issues the MMAs, warps 2-9 run the softmax, two warps per TMEM lane
-// quarter (warp w reads lanes 32 (w % 4) ...), each on 64 of the tile's 128 keys; the two
-// exchange their row maxima through shared memory once per tile.  (Reading the whole row in
+// CTA = (query tile qt, head h, prompt b), 352 threads: warp 0 loads (TMA; lane 0 Q and K,
+// lane 1 V), warp 1 issues the QK MMAs and warp 10 the PV MMAs, warps 2-9 run the softmax, two
+// warps per TMEM lane quarter (warp w reads lanes 32 (w % 4) ...), each on 64 of the tile's
+// 128 keys; the two exchange their row maxima through shared memory once per tile.  (Reading the whole row in
 // both warps instead, to skip the exchange, measured slower.)
 // Shared: Q [3 blocks x 128 rows x 128 B] 48 KB; K ring 2 x (Kh 2 blocks + kr 1 block) 48 KB;
-// V ring 2 x (2 blocks of [128 keys x 64 d]) 32 KB.  TMEM: S0 [0,128), S1 [128,256), O [256,384).
-// Pipeline (MMA issue order): QK0, QK1, PV0, QK2, PV1, QK3, ...; P_j overwrites S_j's first 64
-// columns (bf16 pairs), and QK_{j+2} reuses that buffer only after PV_j in issue order.
+// V ring 2 x (2 blocks of [128 keys x 64 d]) 32 KB.  TMEM: S buffers [0,128), [128,256),
+// [256,384), O [384,512).  Pipeline: QK_j runs up to NSB tiles ahead of the softmax; P_j
+// overwrites S_j's first 64 columns (bf16 pairs), and QK_{j+NSB} reuses that buffer only after
+// PV_j has completed.
 constexpr int AT_Q = 0;
 constexpr int AT_QB = PT * 128;                 // one [128 x 64] bf16 block: 16 KB
 constexpr int AT_K = 3 * AT_QB;                 // 48 KB
@@ -269,13 +335,13 @@ constexpr int AT_V = AT_K + 2 * AT_KS;          // 144 KB
 constexpr int AT_VS = 2 * AT_QB;                // V stage: 32 KB
 constexpr int AT_DATA = AT_V + 2 * AT_VS;       // 208 KB
 constexpr int AT_SMEM = 1024 + AT_DATA + 5120;
-constexpr int AT_THREADS = 320;
+constexpr int AT_THREADS = 352;  // 11 warps
 constexpr int NSB = 3;                             // S buffers in TMEM
 constexpr uint32_t S_COL0 = 0, O_COL = NSB * 128;  // S: [0, 384), O: [384, 512)
 constexpr float kRescaleLog2 = 8.f;  // O is rescaled only when the running max grows by > 2^8
 
 struct __align__(8) AtCtrl {
-    uint64_t q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[NSB], p_ready[NSB], pv_done[NSB], idle;
+    uint64_t q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[NSB], p_ready[NSB], pv_done[NSB], idle[2];
     uint64_t xbar[4][1 + NSB];  // the two softmax warps of a lane quarter meet here: [0] the final row
                                 // sums, [1 + s] the row maxima of S buffer s
     float xmax[NSB][2][128];  // [S buffer][half][row]: row max of each half's raw scores
@@ -323,7 +389,8 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mbar_init(bar(ctrl->p_ready[i]), 8);
             mbar_init(bar(ctrl->pv_done[i]), 1);
         }
-        mbar_init(bar(ctrl->idle), 1);
+        mbar_init(bar(ctrl->idle[0]), 1);
+        mbar_init(bar(ctrl->idle[1]), 1);
         for (int qq = 0; qq < 4; ++qq)
             for (int i = 0; i < 1 + NSB; ++i) mbar_init(bar(ctrl->xbar[qq][i]), 2);
         ctrl->abort = 0;
@@ -376,15 +443,18 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 wait(bar(ctrl->v_full[j & 1]), (uint32_t)(j >> 1) & 1u, &ctrl->never, 1000000000ull);
         }
     } else if (warp == 1) {
-        if (lane == 0) {  // ---- MMA issue ----
+        if (lane == 0) {  // ---- QK issue: S_j = Q K_j^T into S buffer j % NSB ----
             constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
-            constexpr uint32_t idesc_pv = idesc_bf16(128, 128, false, true);
             bool ok = wait(bar(ctrl->q_full), 0u, abort_flag);
-            auto qk = [&](int j) {
-                const int s = j & 1;  // K stage; S buffer j % NSB
-                if (!wait(bar(ctrl->k_full[s]), (uint32_t)(j >> 1) & 1u, abort_flag)) return false;
+            for (int j = 0; ok && j < n_kt; ++j) {
+                const int s = j & 1, sb = j % NSB;  // K stage; S buffer
+                if (!(ok = wait(bar(ctrl->k_full[s]), (uint32_t)(j >> 1) & 1u, abort_flag))) break;
+                if (j >= NSB) {  // the PV that read P_{j-NSB} from this S buffer has completed
+                    const int pj = j - NSB;
+                    if (!(ok = wait(bar(ctrl->pv_done[sb]), (uint32_t)(pj / NSB) & 1u, abort_flag))) break;
+                }
                 tc_fence_after();
-                const uint32_t kb = data_s + AT_K + s * AT_KS, d = tmem + S_COL0 + (j % NSB) * 128;
+                const uint32_t kb = data_s + AT_K + s * AT_KS, d = tmem + S_COL0 + sb * 128;
 #pragma unroll
                 for (int cb = 0; cb < 3; ++cb)
 #pragma unroll
@@ -392,10 +462,19 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         mma_ss(d, sdesc_sw128(data_s + AT_Q + cb * AT_QB + k * 32, 16, 1024),
                                sdesc_sw128(kb + cb * AT_QB + k * 32, 16, 1024), idesc_qk, (cb | k) != 0 ? 1u : 0u);
                 mma_commit(bar(ctrl->k_empty[s]));
-                mma_commit(bar(ctrl->s_full[j % NSB]));
-                return true;
-            };
-            for (int j = 0; ok && j < NSB && j < n_kt; ++j) ok = qk(j);
+                mma_commit(bar(ctrl->s_full[sb]));
+            }
+            if (!ok) *abort_flag = 1;
+            // no MMA of this thread may still run when TMEM is released
+            mma_commit(bar(ctrl->idle[0]));
+            wait(bar(ctrl->idle[0]), 0u, &ctrl->never, 1000000000ull);
+        }
+    } else if (warp == 10) {
+        if (lane == 0) {  // ---- PV issue: O += P_j V_j ----
+            // (A second issuing thread: one thread issues a tcgen05.mma about every 100 clocks,
+            // and the 20 MMAs of a key tile from one thread took longer than the tensor core.)
+            constexpr uint32_t idesc_pv = idesc_bf16(128, 128, false, true);
+            bool ok = true;
             for (int j = 0; ok && j < n_kt; ++j) {
                 const int s = j & 1, sb = j % NSB;
                 if (!(ok = wait(bar(ctrl->p_ready[sb]), (uint32_t)(j / NSB) & 1u, abort_flag))) break;
@@ -408,14 +487,12 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                            (j | kk) != 0 ? 1u : 0u);
                 mma_commit(bar(ctrl->v_empty[s]));
                 mma_commit(bar(ctrl->pv_done[sb]));
-                if (j + NSB < n_kt) ok = qk(j + NSB);
             }
             if (!ok) *abort_flag = 1;
-            // no MMA may still run when TMEM is released
-            mma_commit(bar(ctrl->idle));
-            wait(bar(ctrl->idle), 0u, &ctrl->never, 1000000000ull);
+            mma_commit(bar(ctrl->idle[1]));
+            wait(bar(ctrl->idle[1]), 0u, &ctrl->never, 1000000000ull);
         }
-    } else {  // ---- softmax: warps 2..9, two per TMEM lane quarter, each 64 of the 128 keys ----
+    } else if (warp >= 2 && warp < 10) {  // ---- softmax: two warps per TMEM lane quarter, 64 keys each ----
         const int quarter = warp & 3, half = (warp - 2) >> 2;
         const int row = quarter * 32 + lane;  // query row of the tile = TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -437,7 +514,8 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // keys j*128 + cbase + c with c <= lim are visible (causal, and inside the prompt)
             const int lim = min(qi, L - 1) - j * PT - cbase;
             float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // row max of this warp's raw scores
-            if (__all_sync(0xffffffffu, lim >= 63)) {
+            const bool unmasked = __all_sync(0xffffffffu, lim >= 63);
+            if (unmasked) {
 #pragma unroll
                 for (int c = 0; c < 64; ++c) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(v[c]));
             } else {
@@ -480,18 +558,16 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 tmem_wait_st();
             }
-            const bool live = m_run != -INFINITY;
-            const float nm = -m_run;
-            float sum[4] = {0.f, 0.f, 0.f, 0.f};
+            const bool live = m_run != -INFINITY;  // false only for a row with no visible key yet
+            const float nm = live ? -m_run : 0.f;
             uint32_t pk[32];
+            float psum = unmasked ? softmax_exp<true>(v, scale_log2, nm, pk) : softmax_exp<false>(v, scale_log2, nm, pk);
+            if (!live) {
+                psum = 0.f;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const float p0 = live ? ex2(fmaf(__uint_as_float(v[2 * c]), scale_log2, nm)) : 0.f;
-                const float p1 = live ? ex2(fmaf(__uint_as_float(v[2 * c + 1]), scale_log2, nm)) : 0.f;
-                sum[c & 3] += p0 + p1;
-                pk[c] = pack_bf16x2(p0, p1);
+                for (int c = 0; c < 32; ++c) pk[c] = 0u;
             }
-            l_run += (sum[0] + sum[1]) + (sum[2] + sum[3]);
+            l_run += psum;
             // P over the first 64 columns of this S buffer: keys 2c, 2c+1 in column c
             tmem_st32(lane_base + S_COL0 + s * 128 + half * 32, pk);
             tmem_wait_st();
