@@ -11,15 +11,16 @@
 // running every query in the 576-wide latent space (MQA mode), which pays off only in decode.
 //
 // Three kernels, all in this file:
-//   1. prefill_prep_kernel: Qh[h][t] = [q^C ; RoPE(q^R)] and kr[t] = RoPE(k^R), positions
+//   1. prefill_prep_kernel: Qr[h][t] = RoPE(q^R_{t,h}) and kr[t] = RoPE(k^R_t), positions
 //      t - cu_seqlens[b] (token index within its prompt), rows up to the padded length zeroed.
 //   2. prefill_kv_up_kernel: Kh[h][t] = W^UK_h c_t and Vh[h][t] = W^UV_h c_t, a tcgen05 GEMM
 //      (tile 128 tokens x 256 output columns = 2 heads, K = d_c = 512), bf16 out through TMA.
-//   3. prefill_attn_kernel: causal flash attention per (head, prompt, 128-query tile): S = Q K^T
-//      into TMEM (two buffers), softmax by 4 warps (thread = query row), P written back over S
-//      in TMEM as bf16 and used as the A operand of O += P V (O in TMEM), lazy rescale of O.
+//   3. prefill_attn_kernel: causal flash attention per (head, prompt, 128-query tile): Q = q^C
+//      (read in place from the token-major input by a 4-D TMA map) next to Qr; S = Q K^T into
+//      TMEM (three buffers), softmax by 8 warps (two per query row), P written back over S in
+//      TMEM as bf16 and used as the A operand of O += P V (O in TMEM), lazy rescale of O.
 // Intermediate layouts (workspace, head-major so a (head, 128-token) tile is 128 consecutive
-// rows): Qh [n_h][T_pad][192], Kh, Vh [n_h][T_pad][128], kr [T_pad][64], all bf16;
+// rows): Qr [n_h][T_pad][64], Kh, Vh [n_h][T_pad][128], kr [T_pad][64], all bf16;
 // T_pad = T rounded up to 128.
 #include <math.h>
 
@@ -32,7 +33,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int PDH = 128, PDC = 512, PDR = 64, PDQ = PDH + PDR;  // 192
+constexpr int PDH = 128, PDC = 512, PDR = 64;
 constexpr int PT = 128;                                       // query / key / token tile
 
 // 2^x by the hardware's approximation (relative error about 2^-22, flushes denormals): the
@@ -123,9 +124,8 @@ __device__ __forceinline__ int seq_of(const int32_t *cu, int B, int t) {
 // prompt table once (block 0): cu[0] = 0, non-decreasing, cu[B] = T, every length <= max_len.
 __global__ void __launch_bounds__(256)
 prefill_prep_kernel(int B, const int32_t *__restrict__ cu, int T, int T_pad, int n_h, int max_len,
-                    const __grid_constant__ RopeFreqs rope, const __nv_bfloat16 *__restrict__ q_c,
-                    const __nv_bfloat16 *__restrict__ q_r, const __nv_bfloat16 *__restrict__ k_r,
-                    __nv_bfloat16 *__restrict__ qh, __nv_bfloat16 *__restrict__ kr, unsigned *err) {
+                    const __grid_constant__ RopeFreqs rope, const __nv_bfloat16 *__restrict__ q_r, const __nv_bfloat16 *__restrict__ k_r,
+                    __nv_bfloat16 *__restrict__ qr, __nv_bfloat16 *__restrict__ kr, unsigned *err) {
     const int t = blockIdx.x;
     pdl_trigger();
     pdl_wait();  // the activations may be the previous kernel's output
@@ -143,13 +143,6 @@ prefill_prep_kernel(int B, const int32_t *__restrict__ cu, int T, int T_pad, int
     if (live) pos = t - __ldg(cu + seq_of(cu, B, t));
     if (threadIdx.x < PDR / 2 && live) rope_cos_sin(rope, threadIdx.x, pos, &cs[threadIdx.x], &sn[threadIdx.x]);
     __syncthreads();
-    // q^C: 16 chunks of 8 per head, copied
-    for (int i = threadIdx.x; i < n_h * (PDH / 8); i += blockDim.x) {
-        const int h = i >> 4, c = i & 15;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (live) v = *reinterpret_cast<const uint4 *>(q_c + ((size_t)t * n_h + h) * PDH + c * 8);
-        *reinterpret_cast<uint4 *>(qh + ((size_t)h * T_pad + t) * PDQ + c * 8) = v;
-    }
     // RoPE(q^R): pair k of a head = (x_k, x_{k+32}); thread = (head, k)
     for (int i = threadIdx.x; i < n_h * (PDR / 2); i += blockDim.x) {
         const int h = i >> 5, k = i & 31;
@@ -160,7 +153,7 @@ prefill_prep_kernel(int B, const int32_t *__restrict__ cu, int T, int T_pad, int
             a = x0 * cs[k] - x1 * sn[k];
             b = x1 * cs[k] + x0 * sn[k];
         }
-        __nv_bfloat16 *y = qh + ((size_t)h * T_pad + t) * PDQ + PDH;
+        __nv_bfloat16 *y = qr + ((size_t)h * T_pad + t) * PDR;
         y[k] = __float2bfloat16_rn(a);
         y[k + PDR / 2] = __float2bfloat16_rn(b);
     }
@@ -352,7 +345,8 @@ struct __align__(8) AtCtrl {
 static_assert(sizeof(AtCtrl) <= 5120, "control block");
 
 __global__ void __launch_bounds__(AT_THREADS, 1)
-prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_constant__ CUtensorMap tm_qr,
+                    const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_kr, const __grid_constant__ CUtensorMap tm_v, int B,
                     const int32_t *__restrict__ cu, int T, int T_pad, int n_h, int q_tiles, float scale_log2,
                     __nv_bfloat16 *__restrict__ o, float *__restrict__ lse, unsigned *err) {
@@ -368,7 +362,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     auto bar = [&](uint64_t &x) { return smem_u32(&x); };
 
     pdl_trigger();
-    pdl_wait();  // Qh, Kh, Vh, kr are the previous kernels' output
+    pdl_wait();  // Qr, Kh, Vh, kr are the previous kernels' output (q^C perhaps too)
     // the prompt (clamped to [0, T] so that a bad table cannot move a load or store out of range)
     const int start = min(max(__ldg(cu + b), 0), T);
     const int L = min(max(__ldg(cu + b + 1), start), T) - start;
@@ -406,14 +400,15 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctrl->tmem_base;
-    const int qrow = h * T_pad + start;  // Qh / Kh / Vh row of the prompt's token 0 for this head
+    const int qrow = h * T_pad + start;  // Qr / Kh / Vh row of the prompt's token 0 for this head
 
     if (warp == 0) {
         if (lane == 0) {  // ---- loads: Q, then the K ring (refilled as soon as a QK is done) ----
             bool ok = true;
             int issued = 0;
             mbar_arrive_expect_tx(bar(ctrl->q_full), 3 * AT_QB);
-            tma_load_3d(data_s + AT_Q, &tm_q, 0, qrow + q0, 0, bar(ctrl->q_full));
+            tma_load_4d(data_s + AT_Q, &tm_qc, 0, start + q0, 0, h, bar(ctrl->q_full));  // q^C: blocks 0, 1
+            tma_load_3d(data_s + AT_Q + 2 * AT_QB, &tm_qr, 0, qrow + q0, 0, bar(ctrl->q_full));
             for (int j = 0; j < n_kt; ++j) {
                 const int s = j & 1;
                 if (!(ok = wait(bar(ctrl->k_empty[s]), ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag))) break;
@@ -640,7 +635,7 @@ cudaError_t launch_pdl(void (*kernel)(Exp...), dim3 grid, int threads, int smem,
 }
 
 struct PrefillWs {
-    __nv_bfloat16 *qh, *kh, *vh, *kr;
+    __nv_bfloat16 *qr, *kh, *vh, *kr;
 };
 
 size_t prefill_layout(int n_h, int T_pad, char *base, PrefillWs *w) {
@@ -650,11 +645,11 @@ size_t prefill_layout(int n_h, int T_pad, char *base, PrefillWs *w) {
         off += align_up(bytes, 256);
         return reinterpret_cast<__nv_bfloat16 *>(p);
     };
-    __nv_bfloat16 *qh = take((size_t)n_h * T_pad * PDQ * 2);
+    __nv_bfloat16 *qr = take((size_t)n_h * T_pad * PDR * 2);
     __nv_bfloat16 *kh = take((size_t)n_h * T_pad * PDH * 2);
     __nv_bfloat16 *vh = take((size_t)n_h * T_pad * PDH * 2);
     __nv_bfloat16 *kr = take((size_t)T_pad * PDR * 2);
-    if (w) *w = PrefillWs{qh, kh, vh, kr};
+    if (w) *w = PrefillWs{qr, kh, vh, kr};
     return off;
 }
 
@@ -676,13 +671,14 @@ cudaError_t launch_prefill(const mla_dims_t &d, int B, const int32_t *cu_seqlens
     PrefillWs w;
     if (prefill_layout(d.n_h, T_pad, reinterpret_cast<char *>(ws), &w) > ws_bytes) return cudaErrorInvalidValue;
     const uint64_t hrows = (uint64_t)d.n_h * T_pad;
-    CUtensorMap tm_c, tm_wk, tm_wv, tm_kh, tm_vh, tm_q, tm_k, tm_kr, tm_v;
+    CUtensorMap tm_c, tm_wk, tm_wv, tm_kh, tm_vh, tm_qc, tm_qr, tm_k, tm_kr, tm_v;
     const bool maps = tmap_bf16_colblocks(&tm_c, c_kv, (uint64_t)T, PDC, PDC * 2, PT, 1) &&
                       tmap_bf16_colblocks(&tm_wk, w_uk, (uint64_t)d.n_h * PDH, PDC, PDC * 2, 256, 1) &&
                       tmap_bf16_colblocks(&tm_wv, w_uv, (uint64_t)d.n_h * PDH, PDC, PDC * 2, 256, 1) &&
                       tmap_bf16_colblocks(&tm_kh, w.kh, hrows, PDH, PDH * 2, PT, 2) &&
                       tmap_bf16_colblocks(&tm_vh, w.vh, hrows, PDH, PDH * 2, PT, 2) &&
-                      tmap_bf16_colblocks(&tm_q, w.qh, hrows, PDQ, PDQ * 2, PT, 3) &&
+                      tmap_bf16_head_colblocks(&tm_qc, q_c, (uint64_t)T, (uint64_t)d.n_h, PDH, PT, 2) &&
+                      tmap_bf16_colblocks(&tm_qr, w.qr, hrows, PDR, PDR * 2, PT, 1) &&
                       tmap_bf16_colblocks(&tm_k, w.kh, hrows, PDH, PDH * 2, PT, 2) &&
                       tmap_bf16_colblocks(&tm_kr, w.kr, (uint64_t)T_pad, PDR, PDR * 2, PT, 1) &&
                       tmap_bf16_colblocks(&tm_v, w.vh, hrows, PDH, PDH * 2, PT, 2);
@@ -690,15 +686,16 @@ cudaError_t launch_prefill(const mla_dims_t &d, int B, const int32_t *cu_seqlens
     unsigned *err = device_error_word();
     cudaError_t e = launch_pdl(prefill_prep_kernel, dim3(T_pad), 256, 0, st, B, cu_seqlens, T, T_pad, d.n_h,
                                max_seq_len, make_rope_freqs((double)d.rope_base, d.d_r),
-                               reinterpret_cast<const __nv_bfloat16 *>(q_c), reinterpret_cast<const __nv_bfloat16 *>(q_r),
-                               reinterpret_cast<const __nv_bfloat16 *>(k_r), w.qh, w.kr, err);
+                               reinterpret_cast<const __nv_bfloat16 *>(q_r),
+                               reinterpret_cast<const __nv_bfloat16 *>(k_r), w.qr, w.kr, err);
     if (e != cudaSuccess) return e;
     e = launch_pdl(prefill_kv_up_kernel, dim3(d.n_h / 2, T_pad / PT, 2), 128, UP_SMEM, st, tm_c, tm_wk, tm_wv, tm_kh,
                    tm_vh, T_pad, err);
     if (e != cudaSuccess) return e;
     const int q_tiles = (max_seq_len + PT - 1) / PT;
     const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)(d.d_h + d.d_r)));
-    return launch_pdl(prefill_attn_kernel, dim3(q_tiles, d.n_h, B), AT_THREADS, AT_SMEM, st, tm_q, tm_k, tm_kr, tm_v,
+    return launch_pdl(prefill_attn_kernel, dim3(q_tiles, d.n_h, B), AT_THREADS, AT_SMEM, st, tm_qc, tm_qr, tm_k, tm_kr,
+                      tm_v,
                       B, cu_seqlens, T, T_pad, d.n_h, q_tiles, scale_log2, reinterpret_cast<__nv_bfloat16 *>(o), lse,
                       err);
 }

@@ -51,6 +51,22 @@ inline bool tmap_bf16_colblocks(CUtensorMap *m, const void *base, uint64_t rows,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+// 4-D bf16 map over a token-major tensor [rows][heads][cols] (contiguous): coordinates (x in a
+// 64-wide column block, row, column block, head); a box {64, box_rows, nblk, 1} lands as nblk
+// consecutive [box_rows x 128 B] tiles with 128-byte swizzle: one head's column blocks of
+// box_rows consecutive rows, read in place.
+inline bool tmap_bf16_head_colblocks(CUtensorMap *m, const void *base, uint64_t rows, uint64_t heads, uint64_t cols,
+                                     uint32_t box_rows, uint32_t nblk) {
+    auto fn = tmap_encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[4] = {64, (cuuint64_t)rows, (cuuint64_t)(cols / 64), (cuuint64_t)heads};
+    cuuint64_t gstride[3] = {(cuuint64_t)(heads * cols * 2), 128, (cuuint64_t)(cols * 2)};
+    cuuint32_t box[4] = {64, box_rows, nblk, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), gdim, gstride, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 // 2-D byte map without swizzle: boxes of box_inner bytes x box_rows land row-major.
 inline bool tmap_u8_rows(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t row_bytes,
                          uint32_t box_inner, uint32_t box_rows) {
