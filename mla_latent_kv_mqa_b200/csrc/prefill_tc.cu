@@ -173,10 +173,12 @@ prefill_prep_kernel(int B, const int32_t *__restrict__ cu, int T, int T_pad, int
 
 // ---- 2. K / V reconstruction GEMM -----------------------------------------------------------
 // CTA = (pair of heads, 128-token tile, K or V).  D[t, n] = sum_c c[t, c] W[n0 + n, c]:
-// M = 128 tokens, N = 256 (two heads), K = 512 in 8 chunks of 64 through a 4-stage TMA ring;
+// M = 128 tokens, N = 256 (two heads), K = 512 in 8 chunks of 64 through a 2-stage TMA ring;
 // one thread issues loads and MMAs; the 4 warps move D (TMEM) to a bf16 staging tile in shared
-// memory that one TMA store writes per head.
-constexpr int UP_STAGES = 4;
+// memory that one TMA store writes per head.  ~98 KB of shared memory and 256 TMEM columns,
+// so two CTAs share an SM and one's epilogue overlaps the other's MMAs (measured ~5% fewer
+// cycles per call than one CTA per SM with a 4-stage ring).
+constexpr int UP_STAGES = 2;
 constexpr int UP_A = PT * 128;            // [128 tokens x 64 cols] bf16: 16 KB
 constexpr int UP_B = 256 * 128;           // [256 rows x 64 cols]: 32 KB
 constexpr int UP_STAGE = UP_A + UP_B;     // 48 KB
@@ -190,7 +192,7 @@ struct __align__(8) UpCtrl {
     uint32_t never;  // stays 0: the abort word of drain waits, which must not give up early
 };
 
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(128, 2)
 prefill_kv_up_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_wk,
                      const __grid_constant__ CUtensorMap tm_wv, const __grid_constant__ CUtensorMap tm_kh,
                      const __grid_constant__ CUtensorMap tm_vh, int T_pad, unsigned *err) {
@@ -689,6 +691,7 @@ cudaError_t launch_prefill(const mla_dims_t &d, int B, const int32_t *cu_seqlens
                                reinterpret_cast<const __nv_bfloat16 *>(q_r),
                                reinterpret_cast<const __nv_bfloat16 *>(k_r), w.qr, w.kr, err);
     if (e != cudaSuccess) return e;
+    cudaFuncSetAttribute(prefill_kv_up_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     e = launch_pdl(prefill_kv_up_kernel, dim3(d.n_h / 2, T_pad / PT, 2), 128, UP_SMEM, st, tm_c, tm_wk, tm_wv, tm_kh,
                    tm_vh, T_pad, err);
     if (e != cudaSuccess) return e;
