@@ -299,7 +299,7 @@ mla_status_t mla_decode_project(const mla_dims_t *dims, int B, int s_q, const vo
  *   total_tokens T, the packed token count
  *   max_seq_len  host-side upper bound of the prompt lengths
  *   q_c [T, n_h, d_h], q_r [T, n_h, d_r] (before RoPE), c_kv [T, d_c], k_r [T, d_r] (before
- *                RoPE): bf16, row-major; q_c, c_kv 16-byte aligned
+ *                RoPE): bf16, row-major; q_c, q_r, c_kv 16-byte aligned
  *   w_uk, w_uv   [n_h*d_h, d_c] bf16, 16-byte aligned (written before the call)
  *   workspace    device scratch of workspace_bytes >= mla_prefill_workspace_size(dims, T),
  *                256-byte aligned; its content on entry does not matter

@@ -322,7 +322,7 @@ mla_status_t mla_prefill(const mla_dims_t *dims, int B, const int32_t *cu_seqlen
         return MLA_ERR_INVALID_ARG;
     if (!cu_seqlens || !q_c || !q_r || !c_kv || !k_r || !w_uk || !w_uv || !workspace || !o)
         return MLA_ERR_INVALID_ARG;
-    if (!aligned(q_c, 16) || !aligned(c_kv, 16) || !aligned(w_uk, 16) || !aligned(w_uv, 16) || !aligned(o, 16) ||
+    if (!aligned(q_c, 16) || !aligned(q_r, 16) || !aligned(c_kv, 16) || !aligned(w_uk, 16) || !aligned(w_uv, 16) || !aligned(o, 16) ||
         !aligned(workspace, 256))
         return MLA_ERR_INVALID_ARG;
     if (workspace_bytes < prefill_workspace_bytes(*dims, total_tokens)) return MLA_ERR_WORKSPACE_TOO_SMALL;

@@ -11,16 +11,18 @@
 // running every query in the 576-wide latent space (MQA mode), which pays off only in decode.
 //
 // Three kernels, all in this file:
-//   1. prefill_prep_kernel: Qr[h][t] = RoPE(q^R_{t,h}) and kr[t] = RoPE(k^R_t), positions
-//      t - cu_seqlens[b] (token index within its prompt), rows up to the padded length zeroed.
+//   1. prefill_prep_kernel: the cos / sin table cs[t][k] of each token's position and
+//      kr[t] = RoPE(k^R_t), positions t - cu_seqlens[b] (token index within its prompt), rows up
+//      to the padded length zeroed.
 //   2. prefill_kv_up_kernel: Kh[h][t] = W^UK_h c_t and Vh[h][t] = W^UV_h c_t, a tcgen05 GEMM
 //      (tile 128 tokens x 256 output columns = 2 heads, K = d_c = 512), bf16 out through TMA.
 //   3. prefill_attn_kernel: causal flash attention per (head, prompt, 128-query tile): Q = q^C
-//      (read in place from the token-major input by a 4-D TMA map) next to Qr; S = Q K^T into
+//      (read in place from the token-major input by a 4-D TMA map) next to RoPE(q^R) (rotated
+//      by the softmax warps from q^R and the table on the way into shared memory); S = Q K^T into
 //      TMEM (three buffers), softmax by 8 warps (two per query row), P written back over S in
 //      TMEM as bf16 and used as the A operand of O += P V (O in TMEM), lazy rescale of O.
 // Intermediate layouts (workspace, head-major so a (head, 128-token) tile is 128 consecutive
-// rows): Qr [n_h][T_pad][64], Kh, Vh [n_h][T_pad][128], kr [T_pad][64], all bf16;
+// rows): Kh, Vh [n_h][T_pad][128], kr [T_pad][64], all bf16, and cs [T_pad][32] float2;
 // T_pad = T rounded up to 128.
 #include <math.h>
 
@@ -109,6 +111,10 @@ __device__ __forceinline__ float softmax_exp(const uint32_t (&v)[64], float scal
     return f2lo(a) + f2hi(a);
 }
 
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t v) {
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+
 __device__ __forceinline__ int seq_of(const int32_t *cu, int B, int t) {
     int lo = 0, hi = B;  // largest b with cu[b] <= t
     while (hi - lo > 1) {
@@ -120,17 +126,19 @@ __device__ __forceinline__ int seq_of(const int32_t *cu, int B, int t) {
 }
 
 // ---- 1. prep ----------------------------------------------------------------------------------
-// Block per token row t of [0, T_pad); rows t >= T are written as zeros.  Also checks the
-// prompt table once (block 0): cu[0] = 0, non-decreasing, cu[B] = T, every length <= max_len.
-__global__ void __launch_bounds__(256)
-prefill_prep_kernel(int B, const int32_t *__restrict__ cu, int T, int T_pad, int n_h, int max_len,
-                    const __grid_constant__ RopeFreqs rope, const __nv_bfloat16 *__restrict__ q_r, const __nv_bfloat16 *__restrict__ k_r,
-                    __nv_bfloat16 *__restrict__ qr, __nv_bfloat16 *__restrict__ kr, unsigned *err) {
-    const int t = blockIdx.x;
+// Block = 8 tokens of [0, T_pad), a warp per token, lane k = frequency pair k: the token's
+// cos / sin table row (cs[t][k] = (cos, sin)(pos_t * theta_k), read by the attention kernel to
+// rotate q^R) and kr[t] = RoPE(k^R_t); rows t >= T are written as zeros.  Also checks the prompt
+// table once (block 0): cu[0] = 0, non-decreasing, cu[B] = T, every length <= max_len.
+constexpr int PREP_TOKENS = 8;
+__global__ void __launch_bounds__(32 * PREP_TOKENS)
+prefill_prep_kernel(int B, const int32_t *__restrict__ cu, int T, int max_len, const __grid_constant__ RopeFreqs rope,
+                    const __nv_bfloat16 *__restrict__ k_r, float2 *__restrict__ cs, __nv_bfloat16 *__restrict__ kr,
+                    unsigned *err) {
+    const int t = blockIdx.x * PREP_TOKENS + (threadIdx.x >> 5), k = threadIdx.x & 31;
     pdl_trigger();
     pdl_wait();  // the activations may be the previous kernel's output
-    __shared__ float cs[PDR / 2], sn[PDR / 2];
-    if (t == 0 && threadIdx.x == 0) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
         bool ok = __ldg(cu) == 0 && __ldg(cu + B) == T;
         for (int b = 0; b < B && ok; ++b) {
             const int len = __ldg(cu + b + 1) - __ldg(cu + b);
@@ -138,37 +146,19 @@ prefill_prep_kernel(int B, const int32_t *__restrict__ cu, int T, int T_pad, int
         }
         if (!ok) record_error(err, kErrBadSeqLen);
     }
-    const bool live = t < T;
-    int pos = 0;
-    if (live) pos = t - __ldg(cu + seq_of(cu, B, t));
-    if (threadIdx.x < PDR / 2 && live) rope_cos_sin(rope, threadIdx.x, pos, &cs[threadIdx.x], &sn[threadIdx.x]);
-    __syncthreads();
-    // RoPE(q^R): pair k of a head = (x_k, x_{k+32}); thread = (head, k)
-    for (int i = threadIdx.x; i < n_h * (PDR / 2); i += blockDim.x) {
-        const int h = i >> 5, k = i & 31;
-        float a = 0.f, b = 0.f;
-        if (live) {
-            const __nv_bfloat16 *x = q_r + ((size_t)t * n_h + h) * PDR;
-            const float x0 = __bfloat162float(x[k]), x1 = __bfloat162float(x[k + PDR / 2]);
-            a = x0 * cs[k] - x1 * sn[k];
-            b = x1 * cs[k] + x0 * sn[k];
-        }
-        __nv_bfloat16 *y = qr + ((size_t)h * T_pad + t) * PDR;
-        y[k] = __float2bfloat16_rn(a);
-        y[k + PDR / 2] = __float2bfloat16_rn(b);
+    float c = 0.f, s = 0.f, a = 0.f, b = 0.f;
+    if (t < T) {
+        const int pos = t - __ldg(cu + seq_of(cu, B, t));
+        rope_cos_sin(rope, k, pos, &c, &s);
+        // RoPE pair k = (x_k, x_{k+32})
+        const float x0 = __bfloat162float(k_r[(size_t)t * PDR + k]);
+        const float x1 = __bfloat162float(k_r[(size_t)t * PDR + k + PDR / 2]);
+        a = x0 * c - x1 * s;
+        b = x1 * c + x0 * s;
     }
-    if (threadIdx.x < PDR / 2) {
-        const int k = threadIdx.x;
-        float a = 0.f, b = 0.f;
-        if (live) {
-            const float x0 = __bfloat162float(k_r[(size_t)t * PDR + k]);
-            const float x1 = __bfloat162float(k_r[(size_t)t * PDR + k + PDR / 2]);
-            a = x0 * cs[k] - x1 * sn[k];
-            b = x1 * cs[k] + x0 * sn[k];
-        }
-        kr[(size_t)t * PDR + k] = __float2bfloat16_rn(a);
-        kr[(size_t)t * PDR + k + PDR / 2] = __float2bfloat16_rn(b);
-    }
+    cs[(size_t)t * (PDR / 2) + k] = make_float2(c, s);
+    kr[(size_t)t * PDR + k] = __float2bfloat16_rn(a);
+    kr[(size_t)t * PDR + k + PDR / 2] = __float2bfloat16_rn(b);
 }
 
 // ---- 2. K / V reconstruction GEMM -----------------------------------------------------------
@@ -347,9 +337,9 @@ struct __align__(8) AtCtrl {
 static_assert(sizeof(AtCtrl) <= 5120, "control block");
 
 __global__ void __launch_bounds__(AT_THREADS, 1)
-prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_constant__ CUtensorMap tm_qr,
-                    const __grid_constant__ CUtensorMap tm_k,
+prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_kr, const __grid_constant__ CUtensorMap tm_v, int B,
+                    const __nv_bfloat16 *__restrict__ q_r, const float2 *__restrict__ rope_cs,
                     const int32_t *__restrict__ cu, int T, int T_pad, int n_h, int q_tiles, float scale_log2,
                     __nv_bfloat16 *__restrict__ o, float *__restrict__ lse, unsigned *err) {
     extern __shared__ uint8_t smem_raw[];
@@ -364,7 +354,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_cons
     auto bar = [&](uint64_t &x) { return smem_u32(&x); };
 
     pdl_trigger();
-    pdl_wait();  // Qr, Kh, Vh, kr are the previous kernels' output (q^C perhaps too)
+    pdl_wait();  // Kh, Vh, kr, cs are the previous kernels' output (q^C, q^R perhaps too)
     // the prompt (clamped to [0, T] so that a bad table cannot move a load or store out of range)
     const int start = min(max(__ldg(cu + b), 0), T);
     const int L = min(max(__ldg(cu + b + 1), start), T) - start;
@@ -373,7 +363,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_cons
     const int n_kt = qt + 1;
 
     if (tid == 0) {
-        mbar_init(bar(ctrl->q_full), 1);
+        mbar_init(bar(ctrl->q_full), 9);  // the loader (q^C bytes) and the 8 softmax warps (RoPE(q^R))
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(ctrl->k_full[i]), 1);
             mbar_init(bar(ctrl->k_empty[i]), 1);
@@ -402,15 +392,14 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_cons
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctrl->tmem_base;
-    const int qrow = h * T_pad + start;  // Qr / Kh / Vh row of the prompt's token 0 for this head
+    const int qrow = h * T_pad + start;  // Kh / Vh row of the prompt's token 0 for this head
 
     if (warp == 0) {
         if (lane == 0) {  // ---- loads: Q, then the K ring (refilled as soon as a QK is done) ----
             bool ok = true;
             int issued = 0;
-            mbar_arrive_expect_tx(bar(ctrl->q_full), 3 * AT_QB);
+            mbar_arrive_expect_tx(bar(ctrl->q_full), 2 * AT_QB);
             tma_load_4d(data_s + AT_Q, &tm_qc, 0, start + q0, 0, h, bar(ctrl->q_full));  // q^C: blocks 0, 1
-            tma_load_3d(data_s + AT_Q + 2 * AT_QB, &tm_qr, 0, qrow + q0, 0, bar(ctrl->q_full));
             for (int j = 0; j < n_kt; ++j) {
                 const int s = j & 1;
                 if (!(ok = wait(bar(ctrl->k_empty[s]), ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag))) break;
@@ -496,6 +485,38 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_cons
         const int qi = q0 + row;              // query index within the prompt
         const int cbase = half * 64;          // this warp's key columns of the tile
         const uint32_t xbar0 = bar(ctrl->xbar[quarter][0]);
+        {  // RoPE(q^R) of the tile's rows into Q's column block 2 (rows of 128 B, 128-byte swizzle):
+           // thread = (row r, pairs k0 .. k0 + 15), pair k = (x_k, x_{k+32}) at position q0 + r
+            const int st = tid - 64, r = st >> 1, k0 = (st & 1) * 16;
+            uint32_t ya[8] = {}, yb[8] = {};  // bf16 pairs: elements k0 .. k0+15 and k0+32 .. k0+47
+            if (q0 + r < L) {
+                const size_t t = (size_t)(start + q0 + r);
+                const uint4 *x = reinterpret_cast<const uint4 *>(q_r + (t * n_h + h) * PDR);
+                const float4 *cs = reinterpret_cast<const float4 *>(rope_cs + t * (PDR / 2) + k0);
+                uint32_t xa[8], xb[8];
+                *reinterpret_cast<uint4 *>(xa) = __ldg(x + k0 / 8);
+                *reinterpret_cast<uint4 *>(xa + 4) = __ldg(x + k0 / 8 + 1);
+                *reinterpret_cast<uint4 *>(xb) = __ldg(x + (k0 + 32) / 8);
+                *reinterpret_cast<uint4 *>(xb + 4) = __ldg(x + (k0 + 32) / 8 + 1);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {  // pairs k0 + 2i, k0 + 2i + 1
+                    const float4 q = __ldg(cs + i);  // (cos, sin) of both
+                    const float2 x0 = bf16x2_to_float2(xa[i]), x1 = bf16x2_to_float2(xb[i]);
+                    ya[i] = pack_bf16x2(x0.x * q.x - x1.x * q.y, x0.y * q.z - x1.y * q.w);
+                    yb[i] = pack_bf16x2(x1.x * q.x + x0.x * q.y, x1.y * q.z + x0.y * q.w);
+                }
+            }
+            const uint32_t rowp = data_s + AT_Q + 2 * AT_QB + r * 128;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const int ca = k0 / 8 + c, cb = (k0 + 32) / 8 + c;  // 16-byte chunks of the row
+                st_shared_v4(rowp + ((ca ^ (r & 7)) << 4), ya[4 * c], ya[4 * c + 1], ya[4 * c + 2], ya[4 * c + 3]);
+                st_shared_v4(rowp + ((cb ^ (r & 7)) << 4), yb[4 * c], yb[4 * c + 1], yb[4 * c + 2], yb[4 * c + 3]);
+            }
+            fence_proxy_async_smem();  // visible to the tensor core's reads
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(ctrl->q_full));
+        }
         float m_run = -INFINITY, l_run = 0.f;  // l_run: the sum over this warp's keys
         bool ok = true;
         int j = 0;
@@ -637,7 +658,8 @@ cudaError_t launch_pdl(void (*kernel)(Exp...), dim3 grid, int threads, int smem,
 }
 
 struct PrefillWs {
-    __nv_bfloat16 *qr, *kh, *vh, *kr;
+    float2 *cs;
+    __nv_bfloat16 *kh, *vh, *kr;
 };
 
 size_t prefill_layout(int n_h, int T_pad, char *base, PrefillWs *w) {
@@ -645,13 +667,13 @@ size_t prefill_layout(int n_h, int T_pad, char *base, PrefillWs *w) {
     auto take = [&](size_t bytes) {
         char *p = base ? base + off : nullptr;
         off += align_up(bytes, 256);
-        return reinterpret_cast<__nv_bfloat16 *>(p);
+        return p;
     };
-    __nv_bfloat16 *qr = take((size_t)n_h * T_pad * PDR * 2);
-    __nv_bfloat16 *kh = take((size_t)n_h * T_pad * PDH * 2);
-    __nv_bfloat16 *vh = take((size_t)n_h * T_pad * PDH * 2);
-    __nv_bfloat16 *kr = take((size_t)T_pad * PDR * 2);
-    if (w) *w = PrefillWs{qr, kh, vh, kr};
+    float2 *cs = reinterpret_cast<float2 *>(take((size_t)T_pad * (PDR / 2) * sizeof(float2)));
+    __nv_bfloat16 *kh = reinterpret_cast<__nv_bfloat16 *>(take((size_t)n_h * T_pad * PDH * 2));
+    __nv_bfloat16 *vh = reinterpret_cast<__nv_bfloat16 *>(take((size_t)n_h * T_pad * PDH * 2));
+    __nv_bfloat16 *kr = reinterpret_cast<__nv_bfloat16 *>(take((size_t)T_pad * PDR * 2));
+    if (w) *w = PrefillWs{cs, kh, vh, kr};
     return off;
 }
 
@@ -673,23 +695,21 @@ cudaError_t launch_prefill(const mla_dims_t &d, int B, const int32_t *cu_seqlens
     PrefillWs w;
     if (prefill_layout(d.n_h, T_pad, reinterpret_cast<char *>(ws), &w) > ws_bytes) return cudaErrorInvalidValue;
     const uint64_t hrows = (uint64_t)d.n_h * T_pad;
-    CUtensorMap tm_c, tm_wk, tm_wv, tm_kh, tm_vh, tm_qc, tm_qr, tm_k, tm_kr, tm_v;
+    CUtensorMap tm_c, tm_wk, tm_wv, tm_kh, tm_vh, tm_qc, tm_k, tm_kr, tm_v;
     const bool maps = tmap_bf16_colblocks(&tm_c, c_kv, (uint64_t)T, PDC, PDC * 2, PT, 1) &&
                       tmap_bf16_colblocks(&tm_wk, w_uk, (uint64_t)d.n_h * PDH, PDC, PDC * 2, 256, 1) &&
                       tmap_bf16_colblocks(&tm_wv, w_uv, (uint64_t)d.n_h * PDH, PDC, PDC * 2, 256, 1) &&
                       tmap_bf16_colblocks(&tm_kh, w.kh, hrows, PDH, PDH * 2, PT, 2) &&
                       tmap_bf16_colblocks(&tm_vh, w.vh, hrows, PDH, PDH * 2, PT, 2) &&
                       tmap_bf16_head_colblocks(&tm_qc, q_c, (uint64_t)T, (uint64_t)d.n_h, PDH, PT, 2) &&
-                      tmap_bf16_colblocks(&tm_qr, w.qr, hrows, PDR, PDR * 2, PT, 1) &&
                       tmap_bf16_colblocks(&tm_k, w.kh, hrows, PDH, PDH * 2, PT, 2) &&
                       tmap_bf16_colblocks(&tm_kr, w.kr, (uint64_t)T_pad, PDR, PDR * 2, PT, 1) &&
                       tmap_bf16_colblocks(&tm_v, w.vh, hrows, PDH, PDH * 2, PT, 2);
     if (!maps) return cudaErrorInvalidValue;
     unsigned *err = device_error_word();
-    cudaError_t e = launch_pdl(prefill_prep_kernel, dim3(T_pad), 256, 0, st, B, cu_seqlens, T, T_pad, d.n_h,
-                               max_seq_len, make_rope_freqs((double)d.rope_base, d.d_r),
-                               reinterpret_cast<const __nv_bfloat16 *>(q_r),
-                               reinterpret_cast<const __nv_bfloat16 *>(k_r), w.qr, w.kr, err);
+    cudaError_t e = launch_pdl(prefill_prep_kernel, dim3(T_pad / PREP_TOKENS), 32 * PREP_TOKENS, 0, st, B, cu_seqlens,
+                               T, max_seq_len, make_rope_freqs((double)d.rope_base, d.d_r),
+                               reinterpret_cast<const __nv_bfloat16 *>(k_r), w.cs, w.kr, err);
     if (e != cudaSuccess) return e;
     cudaFuncSetAttribute(prefill_kv_up_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     e = launch_pdl(prefill_kv_up_kernel, dim3(d.n_h / 2, T_pad / PT, 2), 128, UP_SMEM, st, tm_c, tm_wk, tm_wv, tm_kh,
@@ -697,9 +717,8 @@ cudaError_t launch_prefill(const mla_dims_t &d, int B, const int32_t *cu_seqlens
     if (e != cudaSuccess) return e;
     const int q_tiles = (max_seq_len + PT - 1) / PT;
     const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)(d.d_h + d.d_r)));
-    return launch_pdl(prefill_attn_kernel, dim3(q_tiles, d.n_h, B), AT_THREADS, AT_SMEM, st, tm_qc, tm_qr, tm_k, tm_kr,
-                      tm_v,
-                      B, cu_seqlens, T, T_pad, d.n_h, q_tiles, scale_log2, reinterpret_cast<__nv_bfloat16 *>(o), lse,
+    return launch_pdl(prefill_attn_kernel, dim3(q_tiles, d.n_h, B), AT_THREADS, AT_SMEM, st, tm_qc, tm_k, tm_kr,
+                      tm_v, B, reinterpret_cast<const __nv_bfloat16 *>(q_r), static_cast<const float2 *>(w.cs), cu_seqlens, T, T_pad, d.n_h, q_tiles, scale_log2, reinterpret_cast<__nv_bfloat16 *>(o), lse,
                       err);
 }
 

@@ -97,11 +97,12 @@ def test_host_argument_checks(N):
     assert aa(kr=16) == N.MLA_ERR_INVALID_ARG  # a RoPE pool only with the FP8 cache
     assert aa(T_new=0, c_kv=None, T=0, q_c=None) == N.MLA_OK
     # prefill: the supported shape, sizes, null and misaligned pointers, workspace size
-    def pf(B=2, T=256, max_len=128, cu=16, q_c=16, o=16, ws=256, ws_bytes=1 << 40, d=dp):
-        return L.mla_prefill(d, B, cu, T, max_len, q_c, 16, 16, 16, 16, 16, ws, ws_bytes, o, None, None)
+    def pf(B=2, T=256, max_len=128, cu=16, q_c=16, q_r=16, o=16, ws=256, ws_bytes=1 << 40, d=dp):
+        return L.mla_prefill(d, B, cu, T, max_len, q_c, q_r, 16, 16, 16, 16, ws, ws_bytes, o, None, None)
     assert pf(B=0) == N.MLA_OK and pf(T=0) == N.MLA_OK
     assert pf(B=-1) == N.MLA_ERR_INVALID_ARG and pf(max_len=0) == N.MLA_ERR_INVALID_ARG
     assert pf(cu=None) == N.MLA_ERR_INVALID_ARG and pf(q_c=8) == N.MLA_ERR_INVALID_ARG
+    assert pf(q_r=8) == N.MLA_ERR_INVALID_ARG
     assert pf(o=8) == N.MLA_ERR_INVALID_ARG and pf(ws=16) == N.MLA_ERR_INVALID_ARG
     assert pf(ws_bytes=1024) == N.MLA_ERR_WORKSPACE_TOO_SMALL
     assert pf(B=70000) == N.MLA_ERR_INVALID_ARG
