@@ -63,6 +63,22 @@ def test_prefill_sampled_rows_many_tiles(oracle_mod, lens):
     _check(wl, o, lse, oracle_mod, _rows(wl, 4), heads)
 
 
+@pytest.mark.parametrize("lens", [[4096] * 4, [16384]], ids=["bench_4x4096", "one_16384"])
+def test_prefill_full_size_sampled_rows(oracle_mod, lens):
+    """The benchmark's prefill workloads, in the same single mla_prefill call: the last token of
+    every prompt (the longest causal rows), a token on a tile edge and a seeded one, on a few
+    heads (each sampled row costs the oracle a K/V reconstruction over its whole prefix)."""
+    wl = W.make_prefill(88 + len(lens), lens)
+    run = PrefillRun(wl)
+    o, lse = run.run()
+    rng = np.random.default_rng(9)
+    rows = []
+    for b, L in enumerate(wl.seq_lens):
+        rows += [(b, int(L) - 1), (b, 1023), (b, int(rng.integers(0, L)))]
+    heads = rng.choice(128, size=3 if len(lens) > 1 else 2, replace=False)
+    _check(wl, o, lse, oracle_mod, rows, heads)
+
+
 def test_prefill_is_deterministic_and_writes_every_row():
     wl = W.make_prefill(86, [300, 77, 513])
     run = PrefillRun(wl)
