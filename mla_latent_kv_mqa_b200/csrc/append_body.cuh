@@ -28,6 +28,12 @@ AppendArgs append_args(const mla_dims_t &d, int T, const void *c_kv, const void 
 
 // One warp writes token t's cache row.  KV: 0 = f32 cache, 1 = bf16 cache, 2 = fp8 content
 // cache.  Bad sequence indices, positions or block ids are recorded, never dereferenced.
+// The token's inputs depend only on t, so all of a lane's loads (up to AP_BATCH content values
+// and its RoPE pair) are issued before the sequence / position / block-table lookups and travel
+// together with them; loads interleaved with the row's stores would each wait for the previous
+// store (the compiler cannot prove the input and the pool apart), one trip to memory apiece.
+constexpr int AP_BATCH = 16;  // content values per lane in the first batch: d_c <= 512
+
 template <typename Tin, int KV>
 __device__ __forceinline__ void append_token(const AppendArgs &a, const RopeFreqs &rope, int t, int lane,
                                              unsigned *err) {
@@ -39,6 +45,18 @@ __device__ __forceinline__ void append_token(const AppendArgs &a, const RopeFreq
     void *kv_pool = a.kv_pool;
     __nv_bfloat16 *kr_pool = a.kr_pool;
     float *kv_scale = a.kv_scale;
+    const Tin *c_in = c_kv + (size_t)t * d_c;
+    const Tin *k_in = k_r + (size_t)t * d_r;
+    const int half = d_r >> 1;
+
+    float cv[AP_BATCH];
+#pragma unroll
+    for (int i = 0; i < AP_BATCH; ++i) {
+        const int k = lane + 32 * i;
+        cv[i] = k < d_c ? to_f32(c_in[k]) : 0.f;
+    }
+    const float x0 = lane < half ? to_f32(k_in[lane]) : 0.f;
+    const float x1 = lane < half ? to_f32(k_in[lane + half]) : 0.f;
     const int s = seq_idx[t];
     const int p = pos[t];
     if (s < 0 || s >= num_seqs || p < 0 || p / page >= max_blocks) {
@@ -51,17 +69,13 @@ __device__ __forceinline__ void append_token(const AppendArgs &a, const RopeFreq
         return;
     }
     const size_t slot = (size_t)blk * page + (p % page);
-    const Tin *c_in = c_kv + (size_t)t * d_c;
-    const Tin *k_in = k_r + (size_t)t * d_r;
 
     // RoPE of the shared key (pairs k, k + d_r/2).
-    const int half = d_r >> 1;
-    for (int k = lane; k < half; k += 32) {
+    auto put_rope = [&](int k, float a0, float a1) {
         float cs, sn;
         rope_cos_sin(rope, k, p, &cs, &sn);
-        float x0 = to_f32(k_in[k]), x1 = to_f32(k_in[k + half]);
-        float y0 = x0 * cs - x1 * sn;
-        float y1 = x1 * cs + x0 * sn;
+        const float y0 = a0 * cs - a1 * sn;
+        const float y1 = a1 * cs + a0 * sn;
         if (KV == 0) {
             float *row = reinterpret_cast<float *>(kv_pool) + slot * (d_c + d_r) + d_c;
             row[k] = y0;
@@ -75,23 +89,38 @@ __device__ __forceinline__ void append_token(const AppendArgs &a, const RopeFreq
             row[k] = __float2bfloat16_rn(y0);
             row[k + half] = __float2bfloat16_rn(y1);
         }
-    }
+    };
+    if (lane < half) put_rope(lane, x0, x1);
+    for (int k = lane + 32; k < half; k += 32) put_rope(k, to_f32(k_in[k]), to_f32(k_in[k + half]));
 
+    constexpr int kRest = 32 * AP_BATCH;  // content values past the first batch (d_c > 512)
     if (KV == 0) {
         float *row = reinterpret_cast<float *>(kv_pool) + slot * (d_c + d_r);
-        for (int k = lane; k < d_c; k += 32) row[k] = to_f32(c_in[k]);
+#pragma unroll
+        for (int i = 0; i < AP_BATCH; ++i)
+            if (lane + 32 * i < d_c) row[lane + 32 * i] = cv[i];
+        for (int k = kRest + lane; k < d_c; k += 32) row[k] = to_f32(c_in[k]);
     } else if (KV == 1) {
         __nv_bfloat16 *row = reinterpret_cast<__nv_bfloat16 *>(kv_pool) + slot * (d_c + d_r);
-        for (int k = lane; k < d_c; k += 32) row[k] = __float2bfloat16_rn(to_f32(c_in[k]));
+#pragma unroll
+        for (int i = 0; i < AP_BATCH; ++i)
+            if (lane + 32 * i < d_c) row[lane + 32 * i] = __float2bfloat16_rn(cv[i]);
+        for (int k = kRest + lane; k < d_c; k += 32) row[k] = __float2bfloat16_rn(to_f32(c_in[k]));
     } else {
         float amax = 0.f;
-        for (int k = lane; k < d_c; k += 32) amax = fmaxf(amax, fabsf(to_f32(c_in[k])));
+#pragma unroll
+        for (int i = 0; i < AP_BATCH; ++i) amax = fmaxf(amax, fabsf(cv[i]));
+        for (int k = kRest + lane; k < d_c; k += 32) amax = fmaxf(amax, fabsf(to_f32(c_in[k])));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         float sc = 1.f;
         if (amax > 0.f) sc = fmaxf(__fdiv_rn(amax, 448.f), FLT_MIN);
         uint8_t *row = reinterpret_cast<uint8_t *>(kv_pool) + slot * d_c;
-        for (int k = lane; k < d_c; k += 32) {
+#pragma unroll
+        for (int i = 0; i < AP_BATCH; ++i)
+            if (lane + 32 * i < d_c)
+                row[lane + 32 * i] = (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(cv[i], sc), __NV_SATFINITE, __NV_E4M3);
+        for (int k = kRest + lane; k < d_c; k += 32) {
             float x = __fdiv_rn(to_f32(c_in[k]), sc);
             row[k] = (uint8_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
         }
