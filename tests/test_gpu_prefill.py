@@ -79,6 +79,19 @@ def test_prefill_full_size_sampled_rows(oracle_mod, lens):
     _check(wl, o, lse, oracle_mod, rows, heads)
 
 
+def test_prefill_empty_prompts_among_others(oracle_mod):
+    """Zero-length prompts in the table (first, middle, last): their CTAs have no rows and exit,
+    the others are computed as if alone; every row of the call is written."""
+    wl = W.make_prefill(89, [0, 70, 0, 129, 0])
+    run = PrefillRun(wl)
+    o = torch.full((wl.T, 128, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((wl.T, 128), float("nan"), device="cuda")
+    run.run(o, lse)
+    assert bool(torch.isfinite(o.float()).all()) and bool(torch.isfinite(lse).all())
+    rows = [(b, t) for b, L in enumerate(wl.seq_lens) for t in range(L)]
+    _check(wl, o, lse, oracle_mod, rows, np.arange(3, 128, 25))
+
+
 def test_prefill_is_deterministic_and_writes_every_row():
     wl = W.make_prefill(86, [300, 77, 513])
     run = PrefillRun(wl)
