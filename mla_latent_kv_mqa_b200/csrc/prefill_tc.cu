@@ -326,7 +326,7 @@ constexpr uint32_t S_COL0 = 0, O_COL = NSB * 128;  // S: [0, 384), O: [384, 512)
 constexpr float kRescaleLog2 = 8.f;  // O is rescaled only when the running max grows by > 2^8
 
 struct __align__(8) AtCtrl {
-    uint64_t q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[NSB], p_ready[NSB], pv_done[NSB], idle[2];
+    uint64_t q_full, qr_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[NSB], p_ready[NSB], pv_done[NSB], idle[2];
     uint64_t xbar[4][1 + NSB];  // the two softmax warps of a lane quarter meet here: [0] the final row
                                 // sums, [1 + s] the row maxima of S buffer s
     float xmax[NSB][2][128];  // [S buffer][half][row]: row max of each half's raw scores
@@ -363,7 +363,8 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_cons
     const int n_kt = qt + 1;
 
     if (tid == 0) {
-        mbar_init(bar(ctrl->q_full), 9);  // the loader (q^C bytes) and the 8 softmax warps (RoPE(q^R))
+        mbar_init(bar(ctrl->q_full), 1);   // the loader: q^C's bytes
+        mbar_init(bar(ctrl->qr_full), 8);  // the 8 softmax warps: RoPE(q^R)
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(ctrl->k_full[i]), 1);
             mbar_init(bar(ctrl->k_empty[i]), 1);
@@ -432,6 +433,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_cons
         if (lane == 0) {  // ---- QK issue: S_j = Q K_j^T into S buffer j % NSB ----
             constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
             bool ok = wait(bar(ctrl->q_full), 0u, abort_flag);
+            bool qr_in = false;  // the first tile's q^C MMAs go ahead while q^R is being rotated
             for (int j = 0; ok && j < n_kt; ++j) {
                 const int s = j & 1, sb = j % NSB;  // K stage; S buffer
                 if (!(ok = wait(bar(ctrl->k_full[s]), (uint32_t)(j >> 1) & 1u, abort_flag))) break;
@@ -442,11 +444,18 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_cons
                 tc_fence_after();
                 const uint32_t kb = data_s + AT_K + s * AT_KS, d = tmem + S_COL0 + sb * 128;
 #pragma unroll
-                for (int cb = 0; cb < 3; ++cb)
+                for (int cb = 0; cb < 3; ++cb) {
+                    if (cb == 2 && !qr_in) {
+                        if (!(ok = wait(bar(ctrl->qr_full), 0u, abort_flag))) break;
+                        tc_fence_after();
+                        qr_in = true;
+                    }
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
                         mma_ss(d, sdesc_sw128(data_s + AT_Q + cb * AT_QB + k * 32, 16, 1024),
                                sdesc_sw128(kb + cb * AT_QB + k * 32, 16, 1024), idesc_qk, (cb | k) != 0 ? 1u : 0u);
+                }
+                if (!ok) break;
                 mma_commit(bar(ctrl->k_empty[s]));
                 mma_commit(bar(ctrl->s_full[sb]));
             }
@@ -515,7 +524,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_cons
             }
             fence_proxy_async_smem();  // visible to the tensor core's reads
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(ctrl->q_full));
+            if (lane == 0) mbar_arrive(bar(ctrl->qr_full));
         }
         float m_run = -INFINITY, l_run = 0.f;  // l_run: the sum over this warp's keys
         bool ok = true;
