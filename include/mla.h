@@ -217,9 +217,10 @@ mla_status_t mla_decode(const mla_dims_t *dims, int B, int s_q, const void *q_ab
  * mla_decode computes, with the same arguments minus workspace / workspace_bytes.
  *
  * Who it is for: callers that cannot allocate device memory at decode time.  Examples are
- * code running while a CUDA graph is being captured (an allocation there is either illegal
- * or becomes part of the graph) and services with a fixed device-memory budget that is
- * reserved up front.  Instead of a workspace argument, the call uses a scratch array of
+ * services with a fixed device-memory budget that is reserved up front (a decode-time
+ * allocation may fail once that budget is taken), and code on a latency-critical path where
+ * cudaFree / cudaMalloc are not acceptable because they may synchronise the device.
+ * Instead of a workspace argument, the call uses a scratch array of
  * MLA_DECODE_FIXED_SCRATCH_BYTES that lives in the library's own static device storage.
  * It allocates nothing itself.
  *
