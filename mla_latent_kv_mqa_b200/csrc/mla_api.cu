@@ -283,8 +283,11 @@ mla_status_t mla_decode_project(const mla_dims_t *dims, int B, int s_q, const vo
     return mla_out_proj(dims, B * s_q, o_lat, w_uv, o, out_dtype, stream);
 }
 
-// mla_decode on the library's fixed scratch array instead of a caller workspace.  The size
-// check comes first; every other argument is checked by mla_decode itself.  The scratch holds
+// mla_decode on the library's fixed scratch array instead of a caller workspace, for callers
+// that cannot allocate device memory when they decode: a service whose device-memory budget
+// is reserved up front (a late allocation may find none left), or a latency-critical path on
+// which an allocation's possible device synchronisation is not acceptable.  The size check
+// comes first; every other argument is checked by mla_decode itself.  The scratch holds
 // nothing between calls: the decode kernels write every workspace value before they read it.
 mla_status_t mla_decode_fixed_scratch(const mla_dims_t *dims, int B, int s_q, const void *q_abs,
                                       const void *kv_pool, const void *kr_pool,

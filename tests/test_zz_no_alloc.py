@@ -1,6 +1,11 @@
 """mla_decode_fixed_scratch (decode on the library's static scratch array, no caller workspace)
 against mla_decode with a caller workspace, through the C ABI.
 
+The entry point is for callers that cannot allocate device memory when they decode: a service
+whose device-memory budget is reserved up front, where a late allocation may find none left,
+or a latency-critical path on which an allocation's possible device synchronisation is not
+acceptable.
+
 The file name sorts last so that the test also runs after every other test in one session;
 it passes alone in a fresh process as well (the first call on the device does the scratch
 set-up).  Both entry points run the same kernels on the same inputs, so their results must
